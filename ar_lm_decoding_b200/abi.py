@@ -1,0 +1,120 @@
+"""Python binding of libtidar (include/tidar.h): argument marshalling only.
+
+Every function has the name and argument order of its C entry point.  Pointer
+arguments accept a torch tensor (its data_ptr() is passed), a raw integer
+address or None (NULL).  `stream` defaults to torch's current CUDA stream.
+A non-OK status raises TidarError.  There is no fallback: if libtidar.so is
+missing, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtidar.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built: run `python -m ar_lm_decoding_b200.build` "
+                      "(needs nvcc); there is no CPU fallback")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+TIDAR_OK, TIDAR_ERR_INVALID_ARG, TIDAR_ERR_UNSUPPORTED, TIDAR_ERR_WORKSPACE, TIDAR_ERR_CUDA = range(5)
+TIDAR_DEV_BAD_PREFIX, TIDAR_DEV_BAD_TOKEN, TIDAR_DEV_BAD_ACCEPT = 1, 2, 4
+TIDAR_DT_BF16, TIDAR_DT_F32 = 0, 1
+TIDAR_MASK_HYBRID, TIDAR_MASK_CAUSAL = 0, 1
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+_SIGS = {
+    "tidar_attn_workspace_size": (_sz, [_i] * 6),
+    "tidar_attn_step": (_i, [_vp] * 6 + [_i] * 6 + [_f, _i] + [_vp, _vp, _vp, _sz, _vp, _vp]),
+    "tidar_verify_workspace_size": (_sz, [_i] * 3),
+    "tidar_verify": (_i, [_vp, _vp, _i] + [_vp] * 4 + [_i] * 3 + [_vp] * 7 + [_sz, _vp, _vp]),
+    "tidar_kv_commit_workspace_size": (_sz, [_i] * 3),
+    "tidar_kv_commit": (_i, [_vp] * 4 + [_i] * 6 + [_vp] * 4 + [_i, _i, _vp] + [_vp] * 4 + [_sz, _vp, _vp]),
+    "tidar_status_string": (ctypes.c_char_p, [_i]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class TidarError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {tidar_status_string(status)}")
+        self.status = status
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int) -> None:
+    if status != TIDAR_OK:
+        raise TidarError(fn, status)
+
+
+def tidar_status_string(status: int) -> str:
+    return _lib.tidar_status_string(status).decode()
+
+
+def tidar_attn_workspace_size(B, Hq, Hkv, D, k, P_max) -> int:
+    return _lib.tidar_attn_workspace_size(B, Hq, Hkv, D, k, P_max)
+
+
+def tidar_attn_step(q, k_new, v_new, k_cache, v_cache, prefix_len, B, Hq, Hkv, D, k, P_max, softmax_scale,
+                    mask_mode, out, lse, workspace, ws_bytes, dev_status, stream=None) -> None:
+    _check("tidar_attn_step", _lib.tidar_attn_step(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), B, Hq, Hkv, D, k, P_max,
+        softmax_scale, mask_mode, _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def tidar_verify_workspace_size(B, k, V) -> int:
+    return _lib.tidar_verify_workspace_size(B, k, V)
+
+
+def tidar_verify(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u_res, B, k, V, accept_len, resampled,
+                 tokens, n_emitted, logp_d, logq_d, workspace, ws_bytes, dev_status, stream=None) -> None:
+    _check("tidar_verify", _lib.tidar_verify(
+        _ptr(p_logits), _ptr(q_logits), logits_dtype, _ptr(drafts), _ptr(preaccepted), _ptr(u_acc), _ptr(u_res),
+        B, k, V, _ptr(accept_len), _ptr(resampled), _ptr(tokens), _ptr(n_emitted), _ptr(logp_d), _ptr(logq_d),
+        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def tidar_kv_commit_workspace_size(B, k, V) -> int:
+    return _lib.tidar_kv_commit_workspace_size(B, k, V)
+
+
+def tidar_kv_commit(k_caches, v_caches, k_news, v_news, L, B, Hkv, D, k, P_max, prefix_len, accept_len, resampled,
+                    group_logits, logits_dtype, V, u_draft, next_drafts, next_preaccepted, next_q_group, workspace,
+                    ws_bytes, dev_status, stream=None) -> None:
+    _check("tidar_kv_commit", _lib.tidar_kv_commit(
+        _ptr(k_caches), _ptr(v_caches), _ptr(k_news), _ptr(v_news), L, B, Hkv, D, k, P_max, _ptr(prefix_len),
+        _ptr(accept_len), _ptr(resampled), _ptr(group_logits), logits_dtype, V, _ptr(u_draft), _ptr(next_drafts),
+        _ptr(next_preaccepted), _ptr(next_q_group), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def pointer_array(tensors, device):
+    """Device int64 array holding the data pointers of `tensors` (for tidar_kv_commit)."""
+    import torch
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def library_path() -> str:
+    return LIB_PATH

@@ -1,0 +1,169 @@
+// extern "C" entry points of libtidar: host-side argument validation and
+// launch of the device kernels.  Nothing here allocates device memory.
+#include <cmath>
+
+#include "attn.cuh"
+
+namespace tidar {
+size_t verify_workspace_bytes(int B, int k, int V);
+cudaError_t verify_launch(const void *, const void *, int, const int32_t *, const uint8_t *, const float *,
+                          const float *, int, int, int, int32_t *, int32_t *, int32_t *, int32_t *, float *, float *,
+                          void *, int32_t *, cudaStream_t);
+size_t commit_workspace_bytes(int B, int k, int V);
+cudaError_t commit_launch(void *const *, void *const *, const void *const *, const void *const *, int, int, int, int,
+                          int, int, int32_t *, const int32_t *, const int32_t *, const void *, int, int, const float *,
+                          int32_t *, uint8_t *, int32_t *, void *, int32_t *, cudaStream_t);
+
+namespace {
+
+constexpr int kMaxDraft = 16;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+struct AttnPlan {
+    tidar_status status;
+    int R, G, M, Mpad, n_splits;
+    size_t ws_bytes;
+};
+
+AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int k, int P_max) {
+    AttnPlan pl{};
+    if (B < 1 || Hq < 1 || Hkv < 1 || k < 1 || P_max < 0) { pl.status = TIDAR_ERR_INVALID_ARG; return pl; }
+    if (Hq % Hkv != 0 || (D != 64 && D != 128) || k > kMaxDraft) { pl.status = TIDAR_ERR_UNSUPPORTED; return pl; }
+    pl.R = k * (k + 2);
+    pl.G = Hq / Hkv;
+    pl.M = pl.R * pl.G;
+    const int rows = attn_mma_rows_per_tile();
+    const int mtiles = ceil_div(pl.M, rows);
+    pl.Mpad = mtiles * rows;
+    const long base = (long)B * Hkv * mtiles;
+    const int max_splits = std::min(64, ceil_div(P_max + pl.R, 64));
+    long want = (2L * kNumSMs + base - 1) / base;
+    pl.n_splits = (int)std::max(1L, std::min<long>(want, max_splits));
+    const size_t rows_total = (size_t)B * Hkv * pl.n_splits * pl.Mpad;
+    pl.ws_bytes = align256(rows_total * D * sizeof(float)) + align256(rows_total * sizeof(float));
+    pl.status = TIDAR_OK;
+    return pl;
+}
+
+tidar_status launched(cudaError_t e) { return e == cudaSuccess ? TIDAR_OK : TIDAR_ERR_CUDA; }
+
+}  // namespace
+}  // namespace tidar
+
+using namespace tidar;
+
+extern "C" {
+
+size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max) {
+    const AttnPlan pl = plan_attn(B, Hq, Hkv, D, k, P_max);
+    return pl.status == TIDAR_OK ? pl.ws_bytes : 0;
+}
+
+tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new, const void *k_cache,
+                             const void *v_cache, const int32_t *prefix_len, int B, int Hq, int Hkv, int D, int k,
+                             int P_max, float softmax_scale, int mask_mode, void *out, float *lse, void *workspace,
+                             size_t ws_bytes, int32_t *dev_status, void *stream) {
+    const AttnPlan pl = plan_attn(B, Hq, Hkv, D, k, P_max);
+    if (pl.status != TIDAR_OK) return pl.status;
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !prefix_len || !out || !dev_status || !workspace)
+        return TIDAR_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return TIDAR_ERR_INVALID_ARG;
+    if (mask_mode != TIDAR_MASK_HYBRID && mask_mode != TIDAR_MASK_CAUSAL) return TIDAR_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return TIDAR_ERR_INVALID_ARG;
+    if (!aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
+    if (ws_bytes < pl.ws_bytes) return TIDAR_ERR_WORKSPACE;
+    AttnParams p;
+    p.q = static_cast<const bf16 *>(q);
+    p.k_new = static_cast<const bf16 *>(k_new);
+    p.v_new = static_cast<const bf16 *>(v_new);
+    p.k_cache = static_cast<const bf16 *>(k_cache);
+    p.v_cache = static_cast<const bf16 *>(v_cache);
+    p.prefix_len = prefix_len;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.D = D;
+    p.k = k;
+    p.R = pl.R;
+    p.G = pl.G;
+    p.M = pl.M;
+    p.P_max = P_max;
+    p.scale_log2 = softmax_scale * kLog2e;
+    p.mask_mode = mask_mode;
+    p.n_splits = pl.n_splits;
+    p.Mpad = pl.Mpad;
+    const size_t rows_total = (size_t)B * Hkv * pl.n_splits * pl.Mpad;
+    p.part_o = static_cast<float *>(workspace);
+    p.part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows_total * D * sizeof(float)));
+    p.out = static_cast<bf16 *>(out);
+    p.lse = lse;
+    p.dev_status = dev_status;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = attn_mma_launch(p, s);
+    if (e == cudaSuccess) e = attn_combine_launch(p, s);
+    return launched(e);
+}
+
+size_t tidar_verify_workspace_size(int B, int k, int V) {
+    if (B < 1 || k < 1 || k > kMaxDraft || V < 1) return 0;
+    return verify_workspace_bytes(B, k, V);
+}
+
+tidar_status tidar_verify(const void *p_logits, const void *q_logits, int logits_dtype, const int32_t *drafts,
+                          const uint8_t *preaccepted, const float *u_acc, const float *u_res, int B, int k, int V,
+                          int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
+                          float *logp_d, float *logq_d, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                          void *stream) {
+    if (B < 1 || k < 1 || V < 1) return TIDAR_ERR_INVALID_ARG;
+    if (k > kMaxDraft) return TIDAR_ERR_UNSUPPORTED;
+    if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
+    if (!p_logits || !q_logits || !drafts || !preaccepted || !u_acc || !u_res || !accept_len || !resampled ||
+        !tokens || !n_emitted || !workspace || !dev_status)
+        return TIDAR_ERR_INVALID_ARG;
+    if (!aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
+    if (ws_bytes < verify_workspace_bytes(B, k, V)) return TIDAR_ERR_WORKSPACE;
+    return launched(verify_launch(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u_res, B, k, V,
+                                  accept_len, resampled, tokens, n_emitted, logp_d, logq_d, workspace, dev_status,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+size_t tidar_kv_commit_workspace_size(int B, int k, int V) {
+    if (B < 1 || k < 1 || k > kMaxDraft || V < 1) return 0;
+    return commit_workspace_bytes(B, k, V);
+}
+
+tidar_status tidar_kv_commit(void *const *k_caches, void *const *v_caches, const void *const *k_news,
+                             const void *const *v_news, int L, int B, int Hkv, int D, int k, int P_max,
+                             int32_t *prefix_len, const int32_t *accept_len, const int32_t *resampled,
+                             const void *group_logits, int logits_dtype, int V, const float *u_draft,
+                             int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group, void *workspace,
+                             size_t ws_bytes, int32_t *dev_status, void *stream) {
+    if (L < 1 || B < 1 || Hkv < 1 || k < 1 || V < 1 || P_max < 0) return TIDAR_ERR_INVALID_ARG;
+    if (k > kMaxDraft || (D != 64 && D != 128)) return TIDAR_ERR_UNSUPPORTED;
+    if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
+    if (!k_caches || !v_caches || !k_news || !v_news || !prefix_len || !accept_len || !resampled || !group_logits ||
+        !u_draft || !next_drafts || !next_preaccepted || !next_q_group || !workspace || !dev_status)
+        return TIDAR_ERR_INVALID_ARG;
+    if (!aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
+    if (ws_bytes < commit_workspace_bytes(B, k, V)) return TIDAR_ERR_WORKSPACE;
+    return launched(commit_launch(k_caches, v_caches, k_news, v_news, L, B, Hkv, D, k, P_max, prefix_len, accept_len,
+                                  resampled, group_logits, logits_dtype, V, u_draft, next_drafts, next_preaccepted,
+                                  next_q_group, workspace, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+const char *tidar_status_string(tidar_status s) {
+    switch (s) {
+        case TIDAR_OK: return "TIDAR_OK";
+        case TIDAR_ERR_INVALID_ARG: return "TIDAR_ERR_INVALID_ARG";
+        case TIDAR_ERR_UNSUPPORTED: return "TIDAR_ERR_UNSUPPORTED";
+        case TIDAR_ERR_WORKSPACE: return "TIDAR_ERR_WORKSPACE";
+        case TIDAR_ERR_CUDA: return "TIDAR_ERR_CUDA";
+    }
+    return "TIDAR_STATUS_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,27 @@
+// Parameters shared by the attention kernels and the split combine.
+#pragma once
+
+#include "common.cuh"
+
+namespace tidar {
+
+struct AttnParams {
+    const bf16 *q, *k_new, *v_new, *k_cache, *v_cache;
+    const int32_t *prefix_len;
+    int B, Hq, Hkv, D, k, R, G, M, P_max;
+    float scale_log2;  // softmax_scale * log2(e)
+    int mask_mode;
+    int n_splits;      // key ranges per (sequence, KV head)
+    int Mpad;          // M rounded up to the row tile
+    float *part_o;     // [B*Hkv][n_splits][Mpad][D]  normalised partial outputs
+    float *part_lse;   // [B*Hkv][n_splits][Mpad]     natural-log LSE of each range
+    bf16 *out;         // [B, R, Hq, D]
+    float *lse;        // [B, R, Hq] or null
+    int32_t *dev_status;
+};
+
+int attn_mma_rows_per_tile();
+cudaError_t attn_mma_launch(const AttnParams &p, cudaStream_t s);
+cudaError_t attn_combine_launch(const AttnParams &p, cudaStream_t s);
+
+}  // namespace tidar

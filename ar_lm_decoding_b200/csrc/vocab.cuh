@@ -1,0 +1,177 @@
+// Vocabulary-sweep building blocks shared by the verify and the draft
+// selection: per-chunk max / sum-exp statistics with 16-byte loads, and the
+// chunked inverse CDF (sum of non-negative weights, find the chunk, rescan it).
+#pragma once
+
+#include "common.cuh"
+
+namespace tidar {
+
+constexpr int kChunk = 8192;        // vocabulary entries per CTA
+constexpr int kStatThreads = 256;   // kChunk / kStatThreads = 32 entries per thread
+constexpr int kScanThreads = 1024;  // kChunk / kScanThreads = 8 entries per thread
+
+struct ChunkStat {
+    float m;   // max logit of the chunk
+    float pad;
+    double z;  // sum exp(logit - m) over the chunk
+};
+
+__host__ __device__ inline int vocab_chunks(int V) { return (V + kChunk - 1) / kChunk; }
+
+// Load this thread's 32 entries of chunk c of a logit row (missing entries =
+// -inf).  Entry e of thread t is at c*kChunk + (e/8)*2048 + t*8 + e%8 so that a
+// warp reads 512 contiguous bytes (bf16) per step.
+__device__ __forceinline__ void load_chunk32(const void *row, int dtype, int V, int c, float (&v)[32]) {
+    const int tid = threadIdx.x;
+    const int base = c * kChunk;
+    const bool full = base + kChunk <= V;
+    if (dtype == TIDAR_DT_BF16) {
+        const bf16 *r = reinterpret_cast<const bf16 *>(row);
+        const bool aligned = ((reinterpret_cast<uintptr_t>(r) & 15) == 0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i0 = base + j * 2048 + tid * 8;
+            if (full && aligned) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(r + i0));
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[j * 8 + 2 * e] = __uint_as_float(w[e] << 16);
+                    v[j * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[j * 8 + e] = i0 + e < V ? __bfloat162float(r[i0 + e]) : -INFINITY;
+            }
+        }
+    } else {
+        const float *r = reinterpret_cast<const float *>(row);
+        const bool aligned = ((reinterpret_cast<uintptr_t>(r) & 15) == 0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i0 = base + j * 2048 + tid * 8;
+            if (full && aligned) {
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(r + i0));
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(r + i0 + 4));
+                v[j * 8 + 0] = a.x; v[j * 8 + 1] = a.y; v[j * 8 + 2] = a.z; v[j * 8 + 3] = a.w;
+                v[j * 8 + 4] = b.x; v[j * 8 + 5] = b.y; v[j * 8 + 6] = b.z; v[j * 8 + 7] = b.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[j * 8 + e] = i0 + e < V ? r[i0 + e] : -INFINITY;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ int chunk_entry_index(int c, int e) {
+    return c * kChunk + (e >> 3) * 2048 + threadIdx.x * 8 + (e & 7);
+}
+
+// Block-wide max (blockDim.x == kStatThreads).  `red` holds >= 8 floats.
+__device__ __forceinline__ float block_max256(float v, float *red) {
+    v = warp_max(v);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int i = 1; i < kStatThreads / 32; ++i) r = fmaxf(r, red[i]);
+    return r;
+}
+
+// Block-wide sum in double with a fixed order (blockDim.x == nthreads).
+template <int NT>
+__device__ __forceinline__ double block_sum_d(double v, double *red) {
+    v = warp_sum_d(v);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = 0.0;
+#pragma unroll 1
+    for (int i = 0; i < NT / 32; ++i) r += red[i];
+    return r;
+}
+
+// Statistics (max, sum exp) of chunk c of one logit row; every thread returns them.
+__device__ __forceinline__ ChunkStat chunk_stat(const void *row, int dtype, int V, int c, float *redf, double *redd) {
+    float v[32];
+    load_chunk32(row, dtype, V, c, v);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+    mx = block_max256(mx, redf);
+    const float ms = mx * kLog2e;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) s += fast_exp2(fmaf(v[e], kLog2e, -ms));
+    ChunkStat st;
+    st.m = mx;
+    st.pad = 0.f;
+    st.z = block_sum_d<kStatThreads>((double)s, redd);
+    return st;
+}
+
+// Merge chunk statistics in chunk order: returns max m and sum exp(x - m).
+__device__ __forceinline__ void merge_stats(const ChunkStat *st, int n, float &m, double &z) {
+    m = -INFINITY;
+    for (int c = 0; c < n; ++c) m = fmaxf(m, st[c].m);
+    z = 0.0;
+    for (int c = 0; c < n; ++c)
+        if (st[c].m != -INFINITY) z += st[c].z * exp2((double)(st[c].m - m) * 1.4426950408889634);
+}
+
+// Inclusive prefix scan over the kScanThreads x 8 weights of one chunk, then
+// the first local index whose inclusive sum exceeds `target` (or, when
+// rounding leaves none, the last index with positive weight).  `w` holds this
+// thread's 8 consecutive weights (entries tid*8 .. tid*8+7 of the chunk).
+__device__ __forceinline__ int chunk_search(const double (&w)[8], double target, double *scan_buf, int *pick) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    double loc = 0.0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) loc += w[e];
+    // warp inclusive scan of the per-thread totals
+    double incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (tid == 0) { pick[0] = 0x7fffffff; pick[1] = -1; }
+    if (lane == 31) scan_buf[warp] = incl;
+    __syncthreads();
+    if (tid == 0) {
+        double run = 0.0;
+        for (int i = 0; i < kScanThreads / 32; ++i) {
+            const double t = scan_buf[i];
+            scan_buf[i] = run;
+            run += t;
+        }
+    }
+    __syncthreads();
+    double c = scan_buf[warp] + incl - loc;  // exclusive prefix of this thread
+    int first = 0x7fffffff, last = -1;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        c += w[e];
+        if (w[e] > 0.0) {
+            last = tid * 8 + e;
+            if (c > target && first == 0x7fffffff) first = tid * 8 + e;
+        }
+    }
+    if (first != 0x7fffffff) atomicMin(&pick[0], first);
+    if (last >= 0) atomicMax(&pick[1], last);
+    __syncthreads();
+    return pick[0] != 0x7fffffff ? pick[0] : pick[1];
+}
+
+// This thread's 8 consecutive entries (tid*8..tid*8+7) of chunk c as floats (-inf beyond V).
+__device__ __forceinline__ void load_chunk8(const void *row, int dtype, int V, int c, float (&v)[8]) {
+    const int i0 = c * kChunk + threadIdx.x * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = i0 + e < V ? load_logit(row, dtype, (size_t)(i0 + e)) : -INFINITY;
+}
+
+}  // namespace tidar

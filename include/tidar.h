@@ -1,0 +1,200 @@
+/*
+ * tidar.h -- C ABI of the B200 (sm_100a) TiDAR decode-step library.
+ *
+ * One TiDAR decode step ("TiDAR: Think in Diffusion, Talk in Autoregression",
+ * MLSys 2026; awesome-system-papers summary, section 核心方法, "并行
+ * self-speculative 生成 (§3.2)") runs, per layer, a single forward over three
+ * partitions -- the cached causal prefix, the k drafts of the previous step,
+ * and k+1 pre-draft groups of k mask tokens -- then verifies the drafts by AR
+ * rejection sampling, evicts the rejected drafts' KV and takes the next draft
+ * block from the pre-draft group that matches the accept length.
+ *
+ * Three calls cover that hot path:
+ *   tidar_attn_step   the structured hybrid-mask attention of one layer;
+ *   tidar_verify      the AR rejection-sampling verify of the drafts;
+ *   tidar_kv_commit   the exact-KV-cache commit/evict + next-draft selection.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - k = draft length (1..16); R = k(k+2) query rows per sequence.  Rows (and
+ *   the R new keys) are ordered: rows 0..k-1 = drafts d_1..d_k; row
+ *   k + j*k + s = slot s of pre-draft group j (j = 0..k).
+ * - All pointers are DEVICE pointers unless stated otherwise.  The caller owns
+ *   every buffer; the library allocates no device memory, keeps no pointer
+ *   after a call returns and holds no per-call state.
+ * - Every call is asynchronous: it validates its scalar arguments on the host,
+ *   enqueues its kernels on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and returns.  Outputs are valid in stream order.
+ * - Host-side argument errors return TIDAR_ERR_INVALID_ARG (bad pointer or
+ *   size), TIDAR_ERR_UNSUPPORTED (a shape outside the supported set) or
+ *   TIDAR_ERR_WORKSPACE (workspace too small) before anything is launched.
+ *   A failed launch returns TIDAR_ERR_CUDA.
+ * - Data-dependent errors are found on the device: the kernels OR a
+ *   TIDAR_DEV_* bit into *dev_status (an int32 the caller zeroes and reads
+ *   when it chooses) and skip the affected sequence.  No kernel traps, asserts
+ *   or waits without a bound.
+ */
+#ifndef TIDAR_H
+#define TIDAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TIDAR_OK = 0,
+    TIDAR_ERR_INVALID_ARG = 1,
+    TIDAR_ERR_UNSUPPORTED = 2,
+    TIDAR_ERR_WORKSPACE = 3,
+    TIDAR_ERR_CUDA = 4
+} tidar_status;
+
+/* bits of *dev_status */
+#define TIDAR_DEV_BAD_PREFIX 1 /* prefix_len[b] < 0, or beyond the cache capacity */
+#define TIDAR_DEV_BAD_TOKEN 2  /* a draft or resampled token outside [0, V) */
+#define TIDAR_DEV_BAD_ACCEPT 4 /* accept_len[b] outside [0, k] */
+
+typedef enum { TIDAR_DT_BF16 = 0, TIDAR_DT_F32 = 1 } tidar_dtype;
+
+typedef enum {
+    TIDAR_MASK_HYBRID = 0, /* the TiDAR decode mask (below) */
+    TIDAR_MASK_CAUSAL = 1  /* plain causal attention over prefix + R tokens (pure AR mode) */
+} tidar_mask_mode;
+
+/* ------------------------------------------------------------------------ */
+/* Attention                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of workspace tidar_attn_step needs for these sizes (0 if invalid). */
+size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max);
+
+/*
+ * One layer of TiDAR hybrid-mask attention.
+ *
+ * Defined by: TiDAR summary §3.2 (three partitions in one forward; drafts are
+ * verified with this step's causal logits; pre-draft group j is conditioned on
+ * the accept prefix d_1..d_j) and §3.3 (fixed per-step attention pattern over
+ * an exact KV cache); the bxzpzcl.cn walkthrough §1.2 (only the last block is
+ * bidirectional).  Mask for query row r and key n (keys in the order
+ * [cache rows 0..P_b-1 | the R new keys]): every cached key is visible; draft
+ * d_i sees drafts d_1..d_i; a slot of group j sees d_1..d_j and the k slots of
+ * group j; drafts never see mask tokens.  The mask is evaluated from indices.
+ * TIDAR_MASK_CAUSAL instead gives row r the keys 0..P_b+r (the pages' pure
+ * causal likelihood mode).
+ *
+ * q          bf16 [B, R, Hq, D]   post-RoPE queries
+ * k_new      bf16 [B, R, Hkv, D]  post-RoPE keys of this step's R tokens
+ * v_new      bf16 [B, R, Hkv, D]
+ * k_cache    bf16 [B, Hkv, P_max, D]  rows 0..P_b-1 are read, nothing else
+ * v_cache    bf16 [B, Hkv, P_max, D]
+ * prefix_len int32 [B]  P_b, 0 <= P_b <= P_max
+ * Hq % Hkv == 0; query head h reads KV head h / (Hq/Hkv).  D in {64, 128}.
+ * softmax_scale  score multiplier (1/sqrt(D) for the standard scale).
+ * out        bf16 [B, R, Hq, D]  softmax(scale * q k^T) v over the visible keys
+ * lse        f32  [B, R, Hq] or NULL: natural-log log-sum-exp of the scaled scores
+ * workspace  >= tidar_attn_workspace_size(...) bytes of device memory, 256-byte
+ *            aligned; its contents need no initialisation and are clobbered.
+ * dev_status int32*; TIDAR_DEV_BAD_PREFIX set (and that sequence skipped) when
+ *            a prefix length is out of range.
+ * All tensor pointers must be 16-byte aligned.
+ */
+tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new,
+                             const void *k_cache, const void *v_cache, const int32_t *prefix_len,
+                             int B, int Hq, int Hkv, int D, int k, int P_max, float softmax_scale,
+                             int mask_mode, void *out, float *lse, void *workspace, size_t ws_bytes,
+                             int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Verify                                                                    */
+/* ------------------------------------------------------------------------ */
+
+size_t tidar_verify_workspace_size(int B, int k, int V);
+
+/*
+ * AR rejection-sampling verify of the previous step's drafts.
+ *
+ * Defined by: TiDAR summary §3.2 ("Talk": the previous drafts, proposed from
+ * the diffusion marginals, are verified by AR rejection sampling against this
+ * step's causal logits); the speculative-sampling rule it names: draft d_i is
+ * accepted with probability min(1, p_i(d_i)/q_i(d_i)), the scan stops at the
+ * first rejection, and a replacement is drawn from norm(max(0, p - q)) at the
+ * rejected slot.
+ *
+ * p_logits   [B, k, V] (bf16 or f32 per logits_dtype): AR logits for slots
+ *            1..k (slot 1's row is carried from the previous forward; slot i>1
+ *            is the causal output of draft row i-1).  p = softmax(row).
+ * q_logits   [B, k, V]: the stored diffusion logits that proposed the drafts.
+ * drafts     int32 [B, k]; preaccepted uint8 [B]: 1 = slot 1 is the previous
+ *            step's resampled token and is accepted unconditionally.
+ * u_acc      f32 [B, k] uniforms in [0,1): slot i accepted iff u < p(d)/q(d).
+ * u_res      f32 [B]: the residual draw picks the smallest v with
+ *            sum_{w<=v} r(w) > u * sum r, r = max(0, p - q).
+ * accept_len int32 [B]    j* = number of leading accepted slots
+ * resampled  int32 [B]    the residual draw, or -1 when j* = k
+ * tokens     int32 [B, k] tokens emitted this step (accepted drafts that were
+ *            not pre-accepted, then the resampled token), -1 padded
+ * n_emitted  int32 [B]
+ * logp_d, logq_d  f32 [B, k] or NULL: log p_i(d_i), log q_i(d_i)
+ * dev_status TIDAR_DEV_BAD_TOKEN when a draft is outside [0, V).
+ */
+tidar_status tidar_verify(const void *p_logits, const void *q_logits, int logits_dtype,
+                          const int32_t *drafts, const uint8_t *preaccepted,
+                          const float *u_acc, const float *u_res, int B, int k, int V,
+                          int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
+                          float *logp_d, float *logq_d, void *workspace, size_t ws_bytes,
+                          int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Commit                                                                    */
+/* ------------------------------------------------------------------------ */
+
+size_t tidar_kv_commit_workspace_size(int B, int k, int V);
+
+/*
+ * Exact-KV-cache commit/evict plus next-draft selection.
+ *
+ * Defined by: TiDAR summary §3.2 (KV beyond the accept length is evicted, no
+ * recompute) and §3.3 (exact KV cache); the bxzpzcl.cn walkthrough §1.3 (keep
+ * the KV of causally computed accepted tokens, drop rejected tokens' KV at
+ * once, pre-draft tokens never occupy the persistent cache) and §2.2; the
+ * summary's 观察 2 / §3.2 on one-step drafting (each slot drawn independently
+ * from its diffusion marginal) and pre-drafting for every accept outcome.
+ *
+ * For every layer l and sequence b the first accept_len[b] new-key rows (the
+ * accepted drafts, which attended causally, so their K/V equal plain AR K/V)
+ * are copied from k_news[l]/v_news[l] ([B, R, Hkv, D]) into cache rows
+ * P_b .. P_b+j*-1 of k_caches[l]/v_caches[l] ([B, Hkv, P_max, D]); then
+ * prefix_len[b] += j*.  Nothing else in the caches is written.
+ * Next drafts: slot s is the smallest v with sum_{w<=v} softmax(g)(w) > u_draft
+ * [b,s] for g = group_logits[b, j*, s, :]; when j* < k slot 0 is replaced by
+ * resampled[b] and next_preaccepted[b] = 1, else 0.  next_q_group[b] = j*: the
+ * caller's next q_logits are rows group_logits[b, j*, :, :].
+ *
+ * k_caches, v_caches   device array of L device pointers (bf16 caches)
+ * k_news, v_news       device array of L device pointers (bf16 new K/V)
+ * prefix_len           int32 [B], read and updated in place
+ * accept_len, resampled  int32 [B] from tidar_verify
+ * group_logits         [B, k+1, k, V] (bf16 or f32); u_draft f32 [B, k]
+ * next_drafts int32 [B, k]; next_preaccepted uint8 [B]; next_q_group int32 [B]
+ * dev_status  TIDAR_DEV_BAD_ACCEPT / TIDAR_DEV_BAD_PREFIX / TIDAR_DEV_BAD_TOKEN
+ *             when accept_len, P_b + j* or resampled is out of range; that
+ *             sequence is then left untouched.
+ */
+tidar_status tidar_kv_commit(void *const *k_caches, void *const *v_caches,
+                             const void *const *k_news, const void *const *v_news,
+                             int L, int B, int Hkv, int D, int k, int P_max,
+                             int32_t *prefix_len, const int32_t *accept_len, const int32_t *resampled,
+                             const void *group_logits, int logits_dtype, int V, const float *u_draft,
+                             int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group,
+                             void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *tidar_status_string(tidar_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TIDAR_H */

@@ -1,0 +1,129 @@
+"""GPU parity of tidar_attn_step against the CPU oracle (through the C ABI).
+
+Tolerances: output max-abs 2e-2 (bf16), LSE max-abs 1e-4 (fp32 statistics).
+Inputs carry NaN in every cache row at or beyond the prefix length and the
+workspace starts as NaN, so a read outside the visible keys or of an
+unwritten partial shows up as a mismatch.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from ar_lm_decoding_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL = 2e-2, 1e-4
+TINY = synth.CONFIGS["tiny"]
+
+
+def _gpu():
+    import tidar_gpu
+    return tidar_gpu
+
+
+def _check_full(cfg, seed=0, mode=oracle.MASK_HYBRID, inp=None):
+    inp = synth.make_attn_inputs(cfg, seed=seed) if inp is None else inp
+    o_ref, lse_ref, _ = oracle.attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, mode=mode, dense=False)
+    o, lse = _gpu().attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, mode=mode)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    eo = np.abs(o - o_ref).max()
+    el = np.abs(lse - lse_ref).max()
+    assert eo <= O_TOL and el <= LSE_TOL, (cfg.name, eo, el)
+    return o, lse
+
+
+def test_tiny_config():
+    _check_full(TINY)
+
+
+@pytest.mark.parametrize("mode", [oracle.MASK_HYBRID, oracle.MASK_CAUSAL])
+@pytest.mark.parametrize("D", [64, 128])
+def test_modes_and_head_dims(mode, D):
+    _check_full(TINY.with_(D=D, Hq=4, Hkv=2, P=200), seed=1, mode=mode)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 5, 8, 16])
+def test_draft_lengths(k):
+    _check_full(TINY.with_(k=k, P=77, Hq=8, Hkv=2, D=128), seed=k)
+
+
+@pytest.mark.parametrize("P", [0, 1, 63, 64, 65, 300])
+def test_prefix_edges(P):
+    _check_full(TINY.with_(P=P, Hq=4, Hkv=1, D=128), seed=P + 10)
+
+
+def test_ragged_batch():
+    _check_full(TINY.with_(B=5, ragged=(0, 700), Hq=6, Hkv=2, D=128, k=3), seed=3)
+
+
+def test_gqa_groups():
+    for Hq, Hkv in ((8, 1), (12, 2), (32, 8), (5, 5)):
+        _check_full(TINY.with_(Hq=Hq, Hkv=Hkv, P=130, D=128), seed=Hq)
+
+
+def _sample_rows(cfg, inp, n, seed):
+    rng = np.random.default_rng(seed)
+    sb = rng.integers(0, cfg.B, n)
+    sh = rng.integers(0, cfg.Hq, n)
+    sr = rng.integers(0, cfg.R, n)
+    # always include the first and last rows of every partition
+    extra_r = np.array([0, cfg.k - 1, cfg.k, cfg.R - 1])
+    sb = np.concatenate([sb, np.zeros(4, int)])
+    sh = np.concatenate([sh, np.full(4, cfg.Hq - 1)])
+    sr = np.concatenate([sr, extra_r])
+    return sb, sh, sr
+
+
+@pytest.mark.parametrize("name", ["qwen2.5-1.5b_k4", "qwen2.5-1.5b_k16", "qwen3-8b_k8", "qwen3-8b_k8_b8",
+                                  "qwen3-32b_k4", "qwen3-32b_k8", "qwen3-32b_k16"])
+def test_full_size_sampled_rows(name):
+    cfg = synth.CONFIGS[name]
+    inp = synth.make_attn_inputs(cfg, seed=0)
+    o, lse = _gpu().attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    sb, sh, sr = _sample_rows(cfg, inp, 48, seed=1)
+    o_ref, lse_ref = oracle.attn_rows(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, sb, sh, sr)
+    eo = np.abs(o[sb, sr, sh] - o_ref).max()
+    el = np.abs(lse[sb, sr, sh] - lse_ref).max()
+    assert eo <= O_TOL and el <= LSE_TOL, (name, eo, el)
+
+
+def test_group_rows_ignore_later_drafts_bitwise():
+    cfg = TINY.with_(k=4, P=190, Hq=4, Hkv=2)
+    k = cfg.k
+    base = synth.make_attn_inputs(cfg, seed=5)
+    o0, l0 = _gpu().attn(base, cfg.Hq, cfg.Hkv, cfg.D, k)
+    rng = np.random.default_rng(0)
+    for j in range(k + 1):
+        pert = {n: v.copy() for n, v in base.items()}
+        for n in ("k_new", "v_new"):
+            pert[n][:, j:k] = synth.f32_to_bf16_bits(rng.standard_normal(pert[n][:, j:k].shape).astype(np.float32))
+        o1, l1 = _gpu().attn(pert, cfg.Hq, cfg.Hkv, cfg.D, k)
+        rows = slice(k + j * k, k + (j + 1) * k)
+        assert np.array_equal(o0[:, rows], o1[:, rows]) and np.array_equal(l0[:, rows], l1[:, rows])
+    pert = {n: v.copy() for n, v in base.items()}
+    for n in ("k_new", "v_new"):
+        pert[n][:, k:] = synth.f32_to_bf16_bits(rng.standard_normal(pert[n][:, k:].shape).astype(np.float32))
+    o1, l1 = _gpu().attn(pert, cfg.Hq, cfg.Hkv, cfg.D, k)
+    assert np.array_equal(o0[:, :k], o1[:, :k]) and np.array_equal(l0[:, :k], l1[:, :k])
+
+
+def test_deterministic():
+    cfg = synth.CONFIGS["qwen3-8b_k8"].with_(P=1000)
+    inp = synth.make_attn_inputs(cfg, seed=2)
+    a = _gpu().attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k)
+    b = _gpu().attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_bad_prefix_sets_status_and_skips():
+    cfg = TINY.with_(B=2)
+    inp = synth.make_attn_inputs(cfg, seed=4)
+    inp["prefix_len"] = np.array([cfg.P, cfg.P_max + 1], np.int32)
+    o, lse, st = _gpu().attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, want_status=True)
+    assert st & 1
+    assert np.isnan(lse[1]).all()  # the bad sequence is left untouched
+    inp2 = {n: v[:1] if n != "prefix_len" else v[:1] for n, v in inp.items()}
+    o_ref, lse_ref, _ = oracle.attn(inp2, cfg.Hq, cfg.Hkv, cfg.D, cfg.k)
+    assert np.abs(o[0] - o_ref[0]).max() <= O_TOL and np.abs(lse[0] - lse_ref[0]).max() <= LSE_TOL

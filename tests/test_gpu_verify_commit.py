@@ -1,0 +1,167 @@
+"""GPU parity of tidar_verify and tidar_kv_commit against the CPU oracle.
+
+Accept lengths, emitted tokens, resampled tokens, next drafts and committed KV
+must be bit-exact given the same uniforms.  The only exemption: a decision
+whose uniform lies within 1e-5 of the oracle's threshold (|u - p/q| for an
+accept test; the chosen token's normalised CDF interval edge for a draw).
+After an exempt accept decision the oracle is re-run with the GPU's accept
+length forced, so the later outputs are still compared.  Exemptions are
+counted and reported.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from ar_lm_decoding_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+EXEMPT = 1e-5
+
+
+def _gpu():
+    import tidar_gpu
+    return tidar_gpu
+
+
+def _compare_verify(inp, got, report):
+    ref = oracle.verify(inp)
+    B, k = inp["drafts"].shape
+    forced = np.full(B, -1, np.int32)
+    for b in range(B):
+        if got["accept_len"][b] != ref["accept_len"][b]:
+            i = min(got["accept_len"][b], ref["accept_len"][b])  # first slot decided differently
+            margin = abs(float(inp["u_acc"][b, i]) - ref["ratio"][b, i])
+            assert margin < EXEMPT, (b, got["accept_len"][b], ref["accept_len"][b], margin)
+            report.append(("accept", b, margin))
+            forced[b] = got["accept_len"][b]
+    if (forced >= 0).any():
+        ref = oracle.verify(inp, forced_accept_len=forced)
+    assert np.array_equal(got["accept_len"], ref["accept_len"])
+    for b in range(B):
+        if got["resampled"][b] != ref["resampled"][b]:
+            u = float(inp["u_res"][b])
+            margin = min(abs(u - ref["res_lo"][b]), abs(u - ref["res_hi"][b]))
+            assert margin < EXEMPT, (b, got["resampled"][b], ref["resampled"][b], margin)
+            report.append(("resample", b, margin))
+            ref["resampled"][b] = got["resampled"][b]
+            ref["tokens"][b, ref["n_emitted"][b] - 1] = got["resampled"][b]
+    assert np.array_equal(got["resampled"], ref["resampled"])
+    assert np.array_equal(got["n_emitted"], ref["n_emitted"])
+    assert np.array_equal(got["tokens"], ref["tokens"])
+    np.testing.assert_allclose(got["logp_d"], ref["logp_d"], rtol=0, atol=1e-4)
+    np.testing.assert_allclose(got["logq_d"], ref["logq_d"], rtol=0, atol=1e-4)
+    return ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k4", "qwen2.5-1.5b_k16", "qwen3-8b_k8", "qwen3-8b_k8_b8",
+                                  "qwen3-32b_k16"])
+def test_verify_parity(name):
+    cfg = synth.CONFIGS[name]
+    report = []
+    for seed in range(3):
+        inp = synth.make_verify_inputs(cfg, seed=seed)
+        got = _gpu().verify(inp)
+        _compare_verify(inp, got, report)
+    print(f"{name}: exemptions {report}")
+    assert len(report) <= 1
+
+
+def test_verify_many_small_cases():
+    """Many sequences on a small vocabulary: every accept length and the resample path."""
+    report = []
+    rng = np.random.default_rng(0)
+    for V, k, dtype in ((8, 4, "f32"), (1000, 16, "f32"), (9000, 3, "bf16"), (17, 1, "bf16")):
+        B = 256
+        cfg = synth.CONFIGS["tiny"].with_(B=B, V=V, k=k, logits_dtype=dtype, cfg_id=100 + V)
+        inp = synth.make_verify_inputs(cfg, seed=int(rng.integers(1 << 30)))
+        # make p and q close on part of the batch so that long accept runs occur
+        zp = synth.bf16_bits_to_f32(inp["p_logits"]) if dtype == "bf16" else inp["p_logits"].copy()
+        zq = synth.bf16_bits_to_f32(inp["q_logits"]) if dtype == "bf16" else inp["q_logits"].copy()
+        zq[: B // 2] = zp[: B // 2] + 0.1 * rng.standard_normal(zp[: B // 2].shape).astype(np.float32)
+        inp["q_logits"] = synth.f32_to_bf16_bits(zq) if dtype == "bf16" else zq
+        got = _gpu().verify(inp)
+        _compare_verify(inp, got, report)
+        assert len(set(got["accept_len"].tolist())) > 1
+    print(f"exemptions {report}")
+    assert len(report) <= 2
+
+
+def test_verify_bad_draft_sets_status():
+    cfg = synth.CONFIGS["tiny"].with_(B=2)
+    inp = synth.make_verify_inputs(cfg, seed=1)
+    inp["drafts"][1, 2] = cfg.V
+    got = _gpu().verify(inp, want_status=True)
+    assert got["status"] & 2
+    ref = oracle.verify({n: (v[:1] if hasattr(v, "shape") and v.shape[:1] == (2,) else v) for n, v in inp.items()})
+    assert got["accept_len"][0] == ref["accept_len"][0]
+
+
+def _commit_inputs(cfg, seed, L=3):
+    rng = np.random.default_rng(seed)
+    B, k, R, Hkv, D = cfg.B, cfg.k, cfg.R, cfg.Hkv, cfg.D
+    P_max = cfg.P_max
+    kc = rng.integers(0, 2**16, (L, B, Hkv, P_max, D)).astype(np.uint16)
+    vc = rng.integers(0, 2**16, (L, B, Hkv, P_max, D)).astype(np.uint16)
+    kn = rng.integers(0, 2**16, (L, B, R, Hkv, D)).astype(np.uint16)
+    vn = rng.integers(0, 2**16, (L, B, R, Hkv, D)).astype(np.uint16)
+    pl = synth.prefix_lengths(cfg, seed)
+    al = rng.integers(0, k + 1, B).astype(np.int32)
+    rs = np.where(al < k, rng.integers(0, cfg.V, B), -1).astype(np.int32)
+    v = synth.make_verify_inputs(cfg, seed=seed)
+    return kc, vc, kn, vn, pl, al, rs, v["group_logits"], v["u_draft"]
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k4", "qwen3-8b_k8_b8", "qwen2.5-1.5b_k16"])
+def test_commit_parity(name):
+    cfg = synth.CONFIGS[name]
+    report = []
+    for seed in range(2):
+        kc, vc, kn, vn, pl, al, rs, g, ud = _commit_inputs(cfg, seed)
+        got = _gpu().kv_commit(kc, vc, kn, vn, pl, al, rs, g, ud)
+        ref = oracle.kv_commit(kc, vc, kn, vn, pl, al, rs, g, ud)
+        assert np.array_equal(got["k_caches"], ref["k_caches"])
+        assert np.array_equal(got["v_caches"], ref["v_caches"])
+        assert np.array_equal(got["prefix_len"], ref["prefix_len"])
+        assert np.array_equal(got["next_q_group"], ref["next_q_group"])
+        assert np.array_equal(got["next_preaccepted"], ref["next_preaccepted"])
+        diff = got["next_drafts"] != ref["next_drafts"]
+        for b, s in zip(*np.nonzero(diff)):
+            u = float(ud[b, s])
+            margin = min(abs(u - ref["draft_lo"][b, s]), abs(u - ref["draft_hi"][b, s]))
+            assert margin < EXEMPT, (b, s, got["next_drafts"][b, s], ref["next_drafts"][b, s], margin)
+            report.append(("draft", b, s, margin))
+    print(f"{name}: exemptions {report}")
+    assert len(report) <= 1
+
+
+def test_commit_bad_inputs_set_status_and_leave_sequence():
+    cfg = synth.CONFIGS["tiny"].with_(B=3)
+    kc, vc, kn, vn, pl, al, rs, g, ud = _commit_inputs(cfg, 5, L=2)
+    al = np.array([2, cfg.k + 1, 2], np.int32)           # b=1: accept length out of range
+    pl = np.array([cfg.P, cfg.P, cfg.P_max - 1], np.int32)  # b=2: P + j* beyond capacity
+    rs = np.array([3, 3, 3], np.int32)
+    got = _gpu().kv_commit(kc, vc, kn, vn, pl, al, rs, g, ud, want_status=True)
+    assert got["status"] & 4 and got["status"] & 1
+    assert np.array_equal(got["k_caches"][:, 1:], kc[:, 1:])
+    assert list(got["prefix_len"]) == [cfg.P + 2, cfg.P, cfg.P_max - 1]
+    ref = oracle.kv_commit(kc[:, :1], vc[:, :1], kn[:, :1], vn[:, :1], pl[:1], al[:1], rs[:1], g[:1], ud[:1])
+    assert np.array_equal(got["k_caches"][:, :1], ref["k_caches"])
+
+
+def test_step_chain_state_machine():
+    """verify -> commit on the GPU, state handed over as the pages' decode loop does."""
+    cfg = synth.CONFIGS["qwen2.5-1.5b_k4"].with_(B=4, V=30000, ragged=(100, 400))
+    inp = synth.make_verify_inputs(cfg, seed=9)
+    got = _gpu().verify(inp)
+    ref = _compare_verify(inp, got, [])
+    kc, vc, kn, vn, pl, _, _, g, ud = _commit_inputs(cfg, 9, L=2)
+    cg = _gpu().kv_commit(kc, vc, kn, vn, pl, got["accept_len"], got["resampled"], inp["group_logits"],
+                          inp["u_draft"])
+    co = oracle.kv_commit(kc, vc, kn, vn, pl, ref["accept_len"], ref["resampled"], inp["group_logits"],
+                          inp["u_draft"])
+    assert np.array_equal(cg["prefix_len"], pl + got["accept_len"])
+    assert np.array_equal(cg["k_caches"], co["k_caches"])
+    for b in range(cfg.B):
+        if got["accept_len"][b] < cfg.k:
+            assert cg["next_drafts"][b, 0] == got["resampled"][b] and cg["next_preaccepted"][b] == 1
