@@ -34,13 +34,14 @@ AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int k, int P_max) {
     pl.R = k * (k + 2);
     pl.G = Hq / Hkv;
     pl.M = pl.R * pl.G;
-    const int rows = attn_mma_rows_per_tile();
+    const int rows = attn_sm100_rows_per_tile();
+    const int keys = attn_sm100_keys_per_tile();
     const int mtiles = ceil_div(pl.M, rows);
     pl.Mpad = mtiles * rows;
+    // one CTA per SM: split every sequence's key tiles so the grid fills the GPU once
     const long base = (long)B * Hkv * mtiles;
-    const int max_splits = std::min(64, ceil_div(P_max + pl.R, 64));
-    long want = (2L * kNumSMs + base - 1) / base;
-    pl.n_splits = (int)std::max(1L, std::min<long>(want, max_splits));
+    const int max_tiles = ceil_div(P_max, keys) + ceil_div(pl.R, keys);
+    pl.n_splits = (int)std::max(1L, std::min<long>(max_tiles, kNumSMs / base));
     const size_t rows_total = (size_t)B * Hkv * pl.n_splits * pl.Mpad;
     pl.ws_bytes = align256(rows_total * D * sizeof(float)) + align256(rows_total * sizeof(float));
     pl.status = TIDAR_OK;
@@ -103,7 +104,7 @@ tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new
     p.lse = lse;
     p.dev_status = dev_status;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = attn_mma_launch(p, s);
+    cudaError_t e = attn_sm100_launch(p, s);
     if (e == cudaSuccess) e = attn_combine_launch(p, s);
     return launched(e);
 }

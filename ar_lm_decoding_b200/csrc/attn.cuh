@@ -20,8 +20,9 @@ struct AttnParams {
     int32_t *dev_status;
 };
 
-int attn_mma_rows_per_tile();
-cudaError_t attn_mma_launch(const AttnParams &p, cudaStream_t s);
+int attn_sm100_rows_per_tile();
+int attn_sm100_keys_per_tile();
+cudaError_t attn_sm100_launch(const AttnParams &p, cudaStream_t s);
 cudaError_t attn_combine_launch(const AttnParams &p, cudaStream_t s);
 
 }  // namespace tidar

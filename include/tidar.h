@@ -56,6 +56,7 @@ typedef enum {
 #define TIDAR_DEV_BAD_PREFIX 1 /* prefix_len[b] < 0, or beyond the cache capacity */
 #define TIDAR_DEV_BAD_TOKEN 2  /* a draft or resampled token outside [0, V) */
 #define TIDAR_DEV_BAD_ACCEPT 4 /* accept_len[b] outside [0, k] */
+#define TIDAR_DEV_TIMEOUT 8    /* a bounded on-chip wait expired; the outputs are not valid */
 
 typedef enum { TIDAR_DT_BF16 = 0, TIDAR_DT_F32 = 1 } tidar_dtype;
 
