@@ -23,7 +23,7 @@ bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) =
 
 struct AttnPlan {
     tidar_status status;
-    int R, G, M, Mpad, n_splits;
+    int R, G, M, Mpad, n_splits, mtiles, max_tiles;
     size_t ws_bytes;
 };
 
@@ -38,12 +38,11 @@ AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int k, int P_max) {
     const int keys = attn_sm100_keys_per_tile();
     const int mtiles = ceil_div(pl.M, rows);
     pl.Mpad = mtiles * rows;
-    // one CTA per SM: split every sequence's key tiles so the grid fills the GPU once
-    const long base = (long)B * Hkv * mtiles;
-    const int max_tiles = ceil_div(P_max, keys) + ceil_div(pl.R, keys);
-    pl.n_splits = (int)std::max(1L, std::min<long>(max_tiles, kNumSMs / base));
-    const size_t rows_total = (size_t)B * Hkv * pl.n_splits * pl.Mpad;
-    pl.ws_bytes = align256(rows_total * D * sizeof(float)) + align256(rows_total * sizeof(float));
+    pl.mtiles = mtiles;
+    pl.max_tiles = ceil_div(P_max, keys) + ceil_div(pl.R, keys);
+    pl.n_splits = 0;  // chosen at launch (needs the device's cluster occupancy)
+    // one partial-row record (D fp16 + 16 bytes) per row of every split, sized for the largest cluster
+    pl.ws_bytes = align256((size_t)B * Hkv * mtiles * attn_sm100_max_splits() * rows * (2 * D + 16));
     pl.status = TIDAR_OK;
     return pl;
 }
@@ -74,7 +73,7 @@ tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new
         !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
         return TIDAR_ERR_INVALID_ARG;
     if (mask_mode != TIDAR_MASK_HYBRID && mask_mode != TIDAR_MASK_CAUSAL) return TIDAR_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale)) return TIDAR_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f)) return TIDAR_ERR_INVALID_ARG;
     if (!aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
     if (ws_bytes < pl.ws_bytes) return TIDAR_ERR_WORKSPACE;
     AttnParams p;
@@ -95,18 +94,16 @@ tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new
     p.P_max = P_max;
     p.scale_log2 = softmax_scale * kLog2e;
     p.mask_mode = mask_mode;
-    p.n_splits = pl.n_splits;
+    // one CTA per SM: every row tile's key tiles are split over a cluster of CTAs so that the whole
+    // grid is resident in one wave
+    p.n_splits = attn_sm100_pick_splits(D, (long)B * Hkv * pl.mtiles, pl.max_tiles);
     p.Mpad = pl.Mpad;
-    const size_t rows_total = (size_t)B * Hkv * pl.n_splits * pl.Mpad;
-    p.part_o = static_cast<float *>(workspace);
-    p.part_lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + align256(rows_total * D * sizeof(float)));
+    p.part = static_cast<float *>(workspace);
     p.out = static_cast<bf16 *>(out);
     p.lse = lse;
     p.dev_status = dev_status;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = attn_sm100_launch(p, s);
-    if (e == cudaSuccess) e = attn_combine_launch(p, s);
-    return launched(e);
+    return launched(attn_sm100_launch(p, s));
 }
 
 size_t tidar_verify_workspace_size(int B, int k, int V) {

@@ -11,10 +11,9 @@ struct AttnParams {
     int B, Hq, Hkv, D, k, R, G, M, P_max;
     float scale_log2;  // softmax_scale * log2(e)
     int mask_mode;
-    int n_splits;      // key ranges per (sequence, KV head)
+    int n_splits;      // key ranges per (sequence, KV head, row tile): the cluster size
     int Mpad;          // M rounded up to the row tile
-    float *part_o;     // [B*Hkv][n_splits][Mpad][D]  normalised partial outputs
-    float *part_lse;   // [B*Hkv][n_splits][Mpad]     natural-log LSE of each range
+    float *part;       // [B*Hkv*Mpad/128][n_splits][128] partial-row records of 2D+16 bytes (workspace)
     bf16 *out;         // [B, R, Hq, D]
     float *lse;        // [B, R, Hq] or null
     int32_t *dev_status;
@@ -22,7 +21,8 @@ struct AttnParams {
 
 int attn_sm100_rows_per_tile();
 int attn_sm100_keys_per_tile();
+int attn_sm100_pick_splits(int D, long groups, int max_tiles);
+int attn_sm100_max_splits();
 cudaError_t attn_sm100_launch(const AttnParams &p, cudaStream_t s);
-cudaError_t attn_combine_launch(const AttnParams &p, cudaStream_t s);
 
 }  // namespace tidar

@@ -20,13 +20,20 @@
 //               runs its exponentials.  The mask is evaluated from indices;
 //               O is rescaled only when the running max grows by more than
 //               2^8 (a stale max is exact as long as p <= 2^8 fits).
-//   warps 2-3   help load Q, then idle.
+//   warps 2-3   load Q when its rows cannot come through TMA, then idle.
 // TMEM (512 columns): warpgroup w owns S/P at [256w, 256w+128) and O at
 // [256w+128, 256w+128+D).  P (bf16) overwrites the first 64 columns of S; the
 // next S into those columns is issued after the PV that reads P, and
 // tcgen05.mma executes in issue order.
-// At the end the two warpgroups merge their (m, l, O) through shared memory
-// and write the normalised partial output and its LSE for the split combine.
+// The CTAs that split one row tile's keys form a thread-block cluster.  At the
+// end the two warpgroups merge their states through shared memory (each
+// takes half of the columns) into one normalised partial row per query row,
+// stored as fp16 with a per-half-row fp32 scale (|error| <= 2^-12 of the row
+// maximum) and its log2 LSE in fp32; the CTA copies these records, coalesced,
+// to an L2-resident workspace.  After a cluster barrier (the only cross-CTA
+// wait, a hardware barrier) each CTA merges its slice of rows over the
+// cluster's S partials (LSE weights, fixed order) and writes the final bf16
+// output and LSE.
 //
 // Every wait is bounded (clock64 budget); on expiry the CTA raises
 // TIDAR_DEV_TIMEOUT in dev_status, drains, frees TMEM and returns.
@@ -50,11 +57,19 @@ struct Smem {
     static constexpr int STAGE = 2 * KV_TILE;
     static constexpr int KV_OFF = Q_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
-    static constexpr int NBARS = 2 * STAGES + 6;  // kv_full, kv_empty, s_full[2], p_full[2], o_done[2]
+    static constexpr int NBARS = 2 * STAGES + 7;  // kv_full, kv_empty, s_full[2], p_full[2], o_done[2], q_full
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int ALLOC = TOTAL + 1024;  // alignment slack
 };
+
+// Bit i set iff key base+i lies in [a, b) (i = 0..31).
+__device__ __forceinline__ uint32_t range_bits(int a, int b, int base) {
+    const int lo = max(a - base, 0), hi = min(b - base, 32);
+    if (hi <= lo) return 0u;
+    const uint32_t below_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+    return below_hi & ~((1u << lo) - 1u);
+}
 
 // Number of valid keys in tile t (t < TP: prefix tile, else new-key tile).
 __device__ __forceinline__ int tile_valid(int t, int TP, int P, int R) {
@@ -65,7 +80,7 @@ template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_sm100_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_kc,
                       const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
-                      const __grid_constant__ CUtensorMap tm_vn) {
+                      const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_q, int q_tma) {
     using L = Smem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -78,24 +93,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto s_full = [&](int w) { return bar0 + 8u * (2 * STAGES + w); };
     auto p_full = [&](int w) { return bar0 + 8u * (2 * STAGES + 2 + w); };
     auto o_done = [&](int w) { return bar0 + 8u * (2 * STAGES + 4 + w); };
+    const uint32_t q_full = bar0 + 8u * (2 * STAGES + 6);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
     const int split = blockIdx.x, mt = blockIdx.y, bh = blockIdx.z;
     const int b = bh / p.Hkv, kvh = bh % p.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int P = p.prefix_len[b];
-    if (P < 0 || P > p.P_max) {
-        if (tid == 0 && split == 0 && mt == 0) atomicOr(p.dev_status, TIDAR_DEV_BAD_PREFIX);
-        return;
-    }
-    const int TP = ceil_div(P, TN);
-    const int T = TP + ceil_div(p.R, TN);
-    const int t0 = (int)((long)split * T / p.n_splits);
-    const int t1 = (int)((long)(split + 1) * T / p.n_splits);
-    const int n = t1 - t0;
-
-    // ---- set-up ----
+    // ---- set-up that needs nothing from the previous kernel (programmatic dependent launch) ----
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(kv_full(s), 1);
@@ -106,136 +111,195 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mbar_init(p_full(w), 128);
             tc::mbar_init(o_done(w), 1);
         }
+        tc::mbar_init(q_full, q_tma ? 1 : THREADS - 64);
         *abort_flag = 0;
         tc::mbar_fence_init();
-    }
-    if (warp == 0 && lane == 0) {
         tc::tma_prefetch_desc(&tm_kc);
         tc::tma_prefetch_desc(&tm_vc);
         tc::tma_prefetch_desc(&tm_kn);
         tc::tma_prefetch_desc(&tm_vn);
     }
     if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
-    if (warp >= 2) {  // Q tile, K-major with 128-byte swizzle: D/64 blocks of [128 rows][128 B]
-        constexpr int CH = D / 8;
-        for (int idx = tid - 64; idx < TM * CH; idx += THREADS - 64) {
-            const int i = idx / CH, c = idx % CH;
-            const int m = mt * TM + i;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (m < p.M) {
-                const int r = m / p.G, g = m % p.G;
-                v = *reinterpret_cast<const uint4 *>(p.q + ((size_t)(b * p.R + r) * p.Hq + kvh * p.G + g) * D + c * 8);
-            }
-            const int blk = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4 *>(smem + blk * TM * 128 + i * 128 + ((cc ^ (i & 7)) << 4)) = v;
+    // every global read below (prefix lengths, Q, K/V, the workspace) waits for the previous kernel
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    const int P = p.prefix_len[b];
+    if (P < 0 || P > p.P_max) {
+        if (tid == 0 && split == 0 && mt == 0) atomicOr(p.dev_status, TIDAR_DEV_BAD_PREFIX);
+        tc::fence_before_sync();
+        __syncthreads();
+        if (warp == 1) {
+            tc::fence_after_sync();
+            tc::tmem_dealloc(*tmem_slot, 512);
         }
-        tc::fence_proxy_async_smem();
+        return;
+    }
+    const int TP = ceil_div(P, TN);
+    const int T = TP + ceil_div(p.R, TN);
+    const int t0 = (int)((long)split * T / p.n_splits);
+    const int t1 = (int)((long)(split + 1) * T / p.n_splits);
+    const int n = t1 - t0;
+
+    auto issue_tile = [&](int i) {  // K and V of tile i into stage i % STAGES
+        const int st = i % STAGES;
+        tc::mbar_arrive_expect_tx(kv_full(st), L::STAGE);
+        const int t = t0 + i;
+        const uint32_t kd = sKV + st * L::STAGE, vd = kd + L::KV_TILE;
+        if (t < TP) {
+            const int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) {
+                tc::tma_load_2d(kd + h * TN * 128, &tm_kc, h * 64, y, kv_full(st));
+                tc::tma_load_2d(vd + h * TN * 128, &tm_vc, h * 64, y, kv_full(st));
+            }
+        } else {
+            const int z = b * p.R + (t - TP) * TN;
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) {
+                tc::tma_load_3d(kd + h * TN * 128, &tm_kn, h * 64, kvh, z, kv_full(st));
+                tc::tma_load_3d(vd + h * TN * 128, &tm_vn, h * 64, kvh, z, kv_full(st));
+            }
+        }
+    };
+
+    // ---- thread 0 starts the first copies at once ----
+    const int prologue = min(n, STAGES);
+    if (tid == 0) {
+        if (q_tma) {  // rows (r, g) of the tile: box {64 d, G heads, 128/G rows}
+            tc::mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+                tc::tma_load_3d(sQ + h * TM * 128, &tm_q, h * 64, kvh * p.G, b * p.R + mt * (TM / p.G), q_full);
+        }
+        for (int i = 0; i < prologue; ++i) issue_tile(i);
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tbase = *tmem_slot;
-
-    if (warp == 0) {
-        // ================= TMA producer =================
-        if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < n; ++i) {
-                const int st = i % STAGES, u = i / STAGES;
-                if (u > 0 && !tc::mbar_wait(kv_empty(st), (u - 1) & 1, abort_flag, kWaitCycles)) break;
-                tc::mbar_arrive_expect_tx(kv_full(st), L::STAGE);
-                const int t = t0 + i;
-                const uint32_t kd = sKV + st * L::STAGE, vd = kd + L::KV_TILE;
-                if (t < TP) {
-                    const int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) {
-                        tc::tma_load_2d(kd + h * TN * 128, &tm_kc, h * 64, y, kv_full(st));
-                        tc::tma_load_2d(vd + h * TN * 128, &tm_vc, h * 64, y, kv_full(st));
-                    }
-                } else {
-                    const int z = b * p.R + (t - TP) * TN;
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) {
-                        tc::tma_load_3d(kd + h * TN * 128, &tm_kn, h * 64, kvh, z, kv_full(st));
-                        tc::tma_load_3d(vd + h * TN * 128, &tm_vn, h * 64, kvh, z, kv_full(st));
-                    }
-                }
-                issued = i + 1;
+    if (!q_tma && warp >= 2) {  // Q tile, K-major with 128-byte swizzle: D/64 blocks of [128 rows][128 B]
+        constexpr int CH = D / 8;
+        for (int idx = tid - 64; idx < TM * CH; idx += THREADS - 64) {
+            const int i = idx / CH, c = idx % CH;
+            const int m = mt * TM + i;
+            const bf16 *src = p.q;
+            int bytes = 0;
+            if (m < p.M) {
+                const int r = m / p.G, g = m - r * p.G;
+                src = p.q + ((size_t)(b * p.R + r) * p.Hq + kvh * p.G + g) * D + c * 8;
+                bytes = 16;
             }
-            // drain: no copy may land after the CTA exits
-            for (int i = max(0, issued - STAGES); i < issued; ++i)
-                tc::mbar_wait(kv_full(i % STAGES), (i / STAGES) & 1, abort_flag, kWaitCycles);
+            const uint32_t dst = sQ + (c >> 3) * TM * 128 + i * 128 + (((c & 7) ^ (i & 7)) << 4);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+        }
+        asm volatile("cp.async.wait_all;\n" ::: "memory");
+        tc::fence_proxy_async_smem();
+        tc::mbar_arrive(q_full);
+    }
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+        if (warp == 0) {
+            // ================= TMA producer =================
+            if (lane == 0) {
+                int issued = prologue;
+                for (int i = prologue; i < n; ++i) {
+                    const int u = i / STAGES;
+                    if (!tc::mbar_wait(kv_empty(i % STAGES), (u - 1) & 1, abort_flag, kWaitCycles)) break;
+                    issue_tile(i);
+                    issued = i + 1;
+                }
+                // drain: no copy may land after the CTA exits
+                for (int i = max(0, issued - STAGES); i < issued; ++i)
+                    tc::mbar_wait(kv_full(i % STAGES), (i / STAGES) & 1, abort_flag, kWaitCycles);
+            }
+            __syncwarp();
+        } else if (warp == 1) {
+            // ================= MMA issuer =================
+            constexpr uint32_t id_qk = tc::idesc_bf16_f32(TM, TN, 0, 0);
+            constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
+            bool ok = tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);
+            auto issue_qk = [&](int i) {
+                const int st = i % STAGES, w = i & 1;
+                ok = ok && tc::mbar_wait(kv_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
+                if (!ok) return;
+                const int valid = tile_valid(t0 + i, TP, P, p.R);
+                if (valid < TN) {  // keys past the sequence: zero their V rows so that 0 * V stays 0
+                    uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
+                    for (int idx = lane; idx < (TN - valid) * (D / 8); idx += 32) {
+                        const int j = valid + idx / (D / 8), c = idx % (D / 8);
+                        *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    tc::fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    tc::fence_after_sync();
+                    const uint32_t kb = sKV + st * L::STAGE;
+    #pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+                        const uint64_t ad = tc::smem_desc_sw128(sQ + (kk >> 2) * TM * 128 + off, 16, 1024);
+                        const uint64_t bd = tc::smem_desc_sw128(kb + (kk >> 2) * TN * 128 + off, 16, 1024);
+                        tc::mma_ss(tbase + w * 256, ad, bd, id_qk, kk > 0);
+                    }
+                    tc::mma_commit(s_full(w));
+                }
+                __syncwarp();
+            };
+            auto issue_pv = [&](int i) {
+                const int st = i % STAGES, w = i & 1;
+                ok = ok && tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
+                if (!ok) return;
+                if (lane == 0) {
+                    tc::fence_after_sync();
+                    const uint32_t vb = sKV + st * L::STAGE + L::KV_TILE;
+    #pragma unroll
+                    for (int kk = 0; kk < TN / 16; ++kk) {
+                        const uint64_t bd = tc::smem_desc_sw128(vb + kk * 16 * 128, TN * 128, 1024);
+                        tc::mma_ts(tbase + w * 256 + 128, tbase + w * 256 + kk * 8, bd, id_pv, (i >= 2 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(kv_empty(st));
+                    if (i + 2 >= n) tc::mma_commit(o_done(w));
+                }
+                __syncwarp();
+            };
+            if (n > 0) issue_qk(0);
+            if (n > 1) issue_qk(1);
+            for (int i = 0; i < n && ok; ++i) {
+                issue_pv(i);
+                if (i + 2 < n) issue_qk(i + 2);
+            }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ================= MMA issuer =================
-        constexpr uint32_t id_qk = tc::idesc_bf16_f32(TM, TN, 0, 0);
-        constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
-        bool ok = true;
-        auto issue_qk = [&](int i) {
-            const int st = i % STAGES, w = i & 1;
-            ok = ok && tc::mbar_wait(kv_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
-            if (!ok) return;
-            const int valid = tile_valid(t0 + i, TP, P, p.R);
-            if (valid < TN) {  // keys past the sequence: zero their V rows so that 0 * V stays 0
-                uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
-                for (int idx = lane; idx < (TN - valid) * (D / 8); idx += 32) {
-                    const int j = valid + idx / (D / 8), c = idx % (D / 8);
-                    *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
-                        make_uint4(0, 0, 0, 0);
-                }
-                tc::fence_proxy_async_smem();
-            }
-            __syncwarp();
-            if (lane == 0) {
-                tc::fence_after_sync();
-                const uint32_t kb = sKV + st * L::STAGE;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
-                    const uint64_t ad = tc::smem_desc_sw128(sQ + (kk >> 2) * TM * 128 + off, 16, 1024);
-                    const uint64_t bd = tc::smem_desc_sw128(kb + (kk >> 2) * TN * 128 + off, 16, 1024);
-                    tc::mma_ss(tbase + w * 256, ad, bd, id_qk, kk > 0);
-                }
-                tc::mma_commit(s_full(w));
-            }
-            __syncwarp();
-        };
-        auto issue_pv = [&](int i) {
-            const int st = i % STAGES, w = i & 1;
-            ok = ok && tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
-            if (!ok) return;
-            if (lane == 0) {
-                tc::fence_after_sync();
-                const uint32_t vb = sKV + st * L::STAGE + L::KV_TILE;
-#pragma unroll
-                for (int kk = 0; kk < TN / 16; ++kk) {
-                    const uint64_t bd = tc::smem_desc_sw128(vb + kk * 16 * 128, TN * 128, 1024);
-                    tc::mma_ts(tbase + w * 256 + 128, tbase + w * 256 + kk * 8, bd, id_pv, (i >= 2 || kk > 0) ? 1u : 0u);
-                }
-                tc::mma_commit(kv_empty(st));
-                if (i + 2 >= n) tc::mma_commit(o_done(w));
-            }
-            __syncwarp();
-        };
-        if (n > 0) issue_qk(0);
-        if (n > 1) issue_qk(1);
-        for (int i = 0; i < n && ok; ++i) {
-            issue_pv(i);
-            if (i + 2 < n) issue_qk(i + 2);
+        tc::cluster_sync();  // every CTA of the cluster has written its partials
+        if (warp == 1) {
+            tc::fence_after_sync();
+            tc::tmem_dealloc(tbase, 512);
         }
-    } else if (warp >= 4) {
+    } else {
         // ================= softmax warpgroups =================
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
         const int w = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int m_row = mt * TM + row;
         const int r = m_row / p.G;
+        // visible new keys of row r: [0, vis_lim) and [vis_glo, vis_ghi) (same rule as new_key_visible)
+        int vis_lim, vis_glo = 0, vis_ghi = 0;
+        if (p.mask_mode == TIDAR_MASK_CAUSAL || r < p.k) {
+            vis_lim = r + 1;
+        } else {
+            const int grp = (r - p.k) / p.k;
+            vis_lim = grp;
+            vis_glo = p.k + grp * p.k;
+            vis_ghi = vis_glo + p.k;
+        }
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         const uint32_t s_col = tbase + lane_off + w * 256;
         const uint32_t o_col = s_col + 128;
-        float m_run = -INFINITY, l_run = 0.f;
+        const float sl2 = p.scale_log2;  // > 0, so the max of raw scores gives the max of scaled ones
+        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units) and sum
         bool ok = true;
         for (int i = w; i < n; i += 2) {
             if (!tc::mbar_wait(s_full(w), (i >> 1) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
@@ -250,30 +314,36 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             tc::tmem_wait_ld();
             const int t = t0 + i;
-            float mx = -INFINITY;
-            if (t < TP - 1 || (t == TP - 1 && P % TN == 0)) {  // full prefix tile: no mask
-#pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    x[j] *= p.scale_log2;
-                    mx = fmaxf(mx, x[j]);
+            if (t >= TP - 1 && !(t == TP - 1 && P % TN == 0)) {
+                // partial prefix tile (keys beyond P) or new-key tile (the TiDAR mask): visible keys of this
+                // row are [0, lo) and [glo, ghi), all below `end`
+                int lo, glo, ghi, end;
+                if (t < TP) {
+                    lo = end = P - t * TN;
+                    glo = ghi = 0;
+                } else {
+                    const int nn0 = (t - TP) * TN;
+                    lo = vis_lim - nn0;
+                    glo = vis_glo - nn0;
+                    ghi = vis_ghi - nn0;
+                    end = p.R - nn0;
                 }
-            } else if (t < TP) {  // partial prefix tile
-                const int valid = P - t * TN;
+                lo = min(lo, end);
+                ghi = min(ghi, end);
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    x[j] = j < valid ? x[j] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[j]);
-                }
-            } else {  // new-key tile: the TiDAR mask
-                const int nn0 = (t - TP) * TN;
+                for (int c = 0; c < TN / 32; ++c) {
+                    const uint32_t bits = range_bits(0, lo, c * 32) | range_bits(glo, ghi, c * 32);
 #pragma unroll
-                for (int j = 0; j < TN; ++j) {
-                    const int nn = nn0 + j;
-                    const bool vis = nn < p.R && new_key_visible(p.mask_mode, p.k, r, nn);
-                    x[j] = vis ? x[j] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, x[j]);
+                    for (int j = 0; j < 32; ++j) x[c * 32 + j] = (bits >> j) & 1u ? x[c * 32 + j] : -INFINITY;
                 }
             }
+            float mx8[8];  // eight independent chains
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx8[j] = x[j];
+#pragma unroll
+            for (int j = 8; j < TN; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], x[j]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + 8.f;
             if (i >= 2 && __any_sync(0xffffffffu, grow)) {  // rescale O (last written by the PV of tile i-2)
@@ -292,94 +362,185 @@ __global__ void __launch_bounds__(THREADS, 1)
                 l_run *= fast_exp2(m_run - m_new);
                 m_run = m_new;
             }
-            const float m_use = m_run == -INFINITY ? 0.f : m_run;
-            float sum = 0.f;
+            const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+            float sum8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
 #pragma unroll
             for (int c = 0; c < TN / 64; ++c) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float a = fast_exp2(x[c * 64 + 2 * j] - m_use);
-                    const float bb = fast_exp2(x[c * 64 + 2 * j + 1] - m_use);
-                    sum += a + bb;
+                    const float a = fast_exp2(fmaf(x[c * 64 + 2 * j], sl2, neg_m));
+                    const float bb = fast_exp2(fmaf(x[c * 64 + 2 * j + 1], sl2, neg_m));
+                    sum8[(2 * j) & 7] += a;
+                    sum8[(2 * j + 1) & 7] += bb;
                     pk[j] = pack_bf16x2(a, bb);
                 }
                 tc::tmem_st32(s_col + c * 32, pk);
             }
-            l_run += sum;
+            l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(p_full(w));
         }
-        // ---- final O of this warpgroup ----
+        // the next kernel in the stream may launch now: it waits for this grid before touching memory
+        asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+        // ---- merge the two warpgroups (each takes half the columns), then one partial row per CTA ----
         const bool has = n > w;
         if (ok && has) ok = tc::mbar_wait(o_done(w), 0, abort_flag, kWaitCycles);
         tc::fence_after_sync();
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");  // both warpgroups done: the K/V ring is free
-        float *xo = reinterpret_cast<float *>(smem + L::KV_OFF);  // [TM][D + 4] exchange rows
-        float *xm = xo + TM * (D + 4);                              // [TM] m, then [TM] l
-        if (w == 1) {
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");  // both warpgroups' MMAs done: the ring is free
+        constexpr int H = D / 2;     // columns merged by one warpgroup
+        constexpr int HS = H + 4;    // exchange row stride (floats)
+        constexpr int REC = 2 * D + 16;  // partial record: D fp16 values, then lse2, scale[2], pad (bytes)
+        float *xh = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM][HS]: the half the other WG merges
+        float *xml = xh + 2 * TM * HS;                              // [2][2][TM]: m, l
+        uint8_t *rec = reinterpret_cast<uint8_t *>(xml + 4 * TM);   // [TM][REC]
+        const int other = 1 - w;
+        const float m_self = has ? m_run : -INFINITY, l_self = has ? l_run : 0.f;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                if (has && ok) {
-                    tc::tmem_ld32(o_col + c * 32, v);
-                    tc::tmem_wait_ld();
-                } else {
+        for (int c = 0; c < H / 32; ++c) {
+            uint32_t v[32];
+            if (has && ok) {
+                tc::tmem_ld32(o_col + other * H + c * 32, v);
+                tc::tmem_wait_ld();
+            } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 0u;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(xo + row * (D + 4) + c * 32 + j) =
-                        make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                    __uint_as_float(v[j + 3]));
+                for (int j = 0; j < 32; ++j) v[j] = 0u;
             }
-            xm[row] = has ? m_run : -INFINITY;
-            xm[TM + row] = has ? l_run : 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4 *>(xh + (w * TM + row) * HS + c * 32 + j) =
+                    make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                __uint_as_float(v[j + 3]));
+        }
+        xml[(w * 2 + 0) * TM + row] = m_self;
+        xml[(w * 2 + 1) * TM + row] = l_self;
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+        const float m_o = xml[(other * 2 + 0) * TM + row], l_o = xml[(other * 2 + 1) * TM + row];
+        const float mm = fmaxf(m_self, m_o);
+        const float a_s = m_self == -INFINITY ? 0.f : fast_exp2(m_self - mm);
+        const float a_o = m_o == -INFINITY ? 0.f : fast_exp2(m_o - mm);
+        const float lt = l_self * a_s + l_o * a_o;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float f_s = (has && ok) ? a_s * inv : 0.f, f_o = a_o * inv;
+        float hv[H];
+#pragma unroll
+        for (int c = 0; c < H / 32; ++c) {
+            uint32_t v[32];
+            if (has && ok) {
+                tc::tmem_ld32(o_col + w * H + c * 32, v);
+                tc::tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                hv[c * 32 + j] = __uint_as_float(v[j]) * f_s + xh[(other * TM + row) * HS + c * 32 + j] * f_o;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < H; ++j) amax = fmaxf(amax, fabsf(hv[j]));
+        const float scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
+        const float rs = 1.f / scale;
+        uint8_t *myrec = rec + row * REC;
+#pragma unroll
+        for (int j = 0; j < H; j += 8) {
+            uint4 u;
+            u.x = pack_half2(hv[j] * rs, hv[j + 1] * rs);
+            u.y = pack_half2(hv[j + 2] * rs, hv[j + 3] * rs);
+            u.z = pack_half2(hv[j + 4] * rs, hv[j + 5] * rs);
+            u.w = pack_half2(hv[j + 6] * rs, hv[j + 7] * rs);
+            *reinterpret_cast<uint4 *>(myrec + (w * H + j) * 2) = u;
+        }
+        float *hdr = reinterpret_cast<float *>(myrec + 2 * D);
+        hdr[1 + w] = scale;
+        if (w == 0) {
+            hdr[0] = lt > 0.f ? mm + __log2f(lt) : -INFINITY;
+            hdr[3] = 0.f;
         }
         asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        if (w == 0) {
-            const float m0 = has ? m_run : -INFINITY, l0 = has ? l_run : 0.f;
-            const float m1 = xm[row], l1 = xm[TM + row];
-            const float mm = fmaxf(m0, m1);
-            const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
-            const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
-            const float l = l0 * a0 + l1 * a1;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const size_t prow = (size_t)(bh * p.n_splits + split) * p.Mpad + mt * TM + row;
-            float *dst = p.part_o + prow * D;
+        const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
+        const size_t group = (size_t)bh * (p.Mpad / TM) + mt;
+        uint8_t *gbase = reinterpret_cast<uint8_t *>(p.part) + group * S * TM * REC;  // [S][TM][REC]
+        for (int idx = tid - 128; idx < TM * REC / 16; idx += 256)
+            reinterpret_cast<uint4 *>(gbase + (size_t)split * TM * REC)[idx] = reinterpret_cast<const uint4 *>(rec)[idx];
+        __threadfence();
+        tc::fence_before_sync();
+        tc::cluster_sync();
+
+        // ---- merge the S partials of this CTA's slice of rows (L2-resident) ----
+        const int per = ceil_div(TM, S);
+        const int row0 = split * per, nrows = min(TM, row0 + per) - row0;
+        const int wi = warp - 4;  // 8 merging warps
+        constexpr int PER = D / 32;  // columns per lane
+        const int half = (lane * PER) / H;
+        // a warp takes rows wi, wi+8, ...; two at a time with all their records (<= 2 x 8) in flight
+        for (int lr0 = wi; lr0 < nrows; lr0 += 16) {
+            float lsev[2][8], scl[2][8];
+            uint2 raw[2][8];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                if (has && ok) {
-                    tc::tmem_ld32(o_col + c * 32, v);
-                    tc::tmem_wait_ld();
-                } else {
+            for (int j = 0; j < 2; ++j) {
+                const int lr = lr0 + 8 * j;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 0u;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 o1 = *reinterpret_cast<const float4 *>(xo + row * (D + 4) + c * 32 + j);
-                    float4 o;
-                    o.x = (__uint_as_float(v[j]) * a0 + o1.x * a1) * inv;
-                    o.y = (__uint_as_float(v[j + 1]) * a0 + o1.y * a1) * inv;
-                    o.z = (__uint_as_float(v[j + 2]) * a0 + o1.z * a1) * inv;
-                    o.w = (__uint_as_float(v[j + 3]) * a0 + o1.w * a1) * inv;
-                    *reinterpret_cast<float4 *>(dst + c * 32 + j) = o;
+                for (int sp = 0; sp < 8; ++sp) {
+                    lsev[j][sp] = -INFINITY;
+                    if (sp < S && lr < nrows) {
+                        const uint8_t *r0 = gbase + ((size_t)sp * TM + row0 + lr) * REC;
+                        const float *hd = reinterpret_cast<const float *>(r0 + 2 * D);
+                        lsev[j][sp] = __ldcg(hd);
+                        scl[j][sp] = __ldcg(hd + 1 + half);
+                        if constexpr (PER == 4)
+                            raw[j][sp] = __ldcg(reinterpret_cast<const uint2 *>(r0 + lane * PER * 2));
+                        else
+                            raw[j][sp].x = __ldcg(reinterpret_cast<const unsigned int *>(r0 + lane * PER * 2));
+                    }
                 }
             }
-            p.part_lse[prow] = l > 0.f ? (mm + __log2f(l)) * kLn2 : -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int lr = lr0 + 8 * j;
+                const int m = mt * TM + row0 + lr;
+                if (lr >= nrows || m >= p.M) continue;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int sp = 0; sp < 8; ++sp) mx = fmaxf(mx, lsev[j][sp]);
+                float acc[PER], wsum = 0.f;
+#pragma unroll
+                for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+#pragma unroll
+                for (int sp = 0; sp < 8; ++sp) {
+                    if (lsev[j][sp] != -INFINITY) {
+                        const float wq = fast_exp2(lsev[j][sp] - mx);
+                        wsum += wq;
+                        const float f = wq * scl[j][sp];
+                        const float2 v0 = unpack_half2(raw[j][sp].x);
+                        acc[0] += f * v0.x;
+                        acc[1] += f * v0.y;
+                        if constexpr (PER == 4) {
+                            const float2 v1 = unpack_half2(raw[j][sp].y);
+                            acc[2] += f * v1.x;
+                            acc[3] += f * v1.y;
+                        }
+                    }
+                }
+                const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+                const int rq = m / p.G, h = kvh * p.G + (m - rq * p.G);
+                const size_t orow = (size_t)(b * p.R + rq) * p.Hq + h;
+                bf16 *dst = p.out + orow * D + lane * PER;
+                if constexpr (PER == 4) {
+                    uint2 v;
+                    v.x = pack_bf16x2(acc[0] * winv, acc[1] * winv);
+                    v.y = pack_bf16x2(acc[2] * winv, acc[3] * winv);
+                    *reinterpret_cast<uint2 *>(dst) = v;
+                } else {
+                    *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * winv, acc[1] * winv);
+                }
+                if (p.lse && lane == 0) p.lse[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+            }
         }
-    }
-
-    // ---- teardown ----
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 1) {
-        tc::fence_after_sync();
-        tc::tmem_dealloc(tbase, 512);
     }
     if (tid == 0 && *abort_flag) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
 }
@@ -415,28 +576,90 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims
 
 template <int D>
 cudaError_t launch(const AttnParams &p, cudaStream_t s) {
-    CUtensorMap kc, vc, kn, vn;
+    CUtensorMap kc, vc, kn, vn, qm;
     const cuuint64_t dc[2] = {(cuuint64_t)D, (cuuint64_t)p.B * p.Hkv * p.P_max};
     const cuuint64_t sc[1] = {(cuuint64_t)D * 2};
     const cuuint32_t bc[2] = {64, TN};
     const cuuint64_t dn[3] = {(cuuint64_t)D, (cuuint64_t)p.Hkv, (cuuint64_t)p.B * p.R};
     const cuuint64_t sn[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.Hkv * D * 2};
     const cuuint32_t bn[3] = {64, 1, TN};
+    // Q as {D, Hq, B*R}: a box of G heads x 128/G rows is one packed row tile when G divides 128
+    const int q_tma = (TM % p.G == 0) ? 1 : 0;
+    const cuuint64_t dq[3] = {(cuuint64_t)D, (cuuint64_t)p.Hq, (cuuint64_t)p.B * p.R};
+    const cuuint64_t sq[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.Hq * D * 2};
+    const cuuint32_t bq[3] = {64, (cuuint32_t)(q_tma ? p.G : 1), (cuuint32_t)(q_tma ? TM / p.G : 1)};
     if (!make_map(&kc, p.k_cache, 2, dc, sc, bc) || !make_map(&vc, p.v_cache, 2, dc, sc, bc) ||
-        !make_map(&kn, p.k_new, 3, dn, sn, bn) || !make_map(&vn, p.v_new, 3, dn, sn, bn))
+        !make_map(&kn, p.k_new, 3, dn, sn, bn) || !make_map(&vn, p.v_new, 3, dn, sn, bn) ||
+        !make_map(&qm, p.q, 3, dq, sq, bq))
         return cudaErrorInvalidValue;
     const int smem = Smem<D>::ALLOC;
     cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_splits, p.Mpad / TM, p.B * p.Hkv);
-    attn_sm100_kernel<D><<<grid, THREADS, smem, s>>>(p, kc, vc, kn, vn);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_splits, p.Mpad / TM, p.B * p.Hkv);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;  // the splits of one row tile form a cluster
+    attr[0].val.clusterDim.x = p.n_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap set-up with the previous kernel
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, p, kc, vc, kn, vn, qm, q_tma);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// Clusters of `S` CTAs of this kernel that can be resident at once (0 if the query fails).
+template <int D>
+int max_active_clusters(int S) {
+    static int cache[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+    if (cache[S] >= 0) return cache[S];
+    const int smem = Smem<D>::ALLOC;
+    if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_sm100_kernel<D>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cache[S] = n;
+    return n;
 }
 
 }  // namespace
 
 int attn_sm100_rows_per_tile() { return TM; }
 int attn_sm100_keys_per_tile() { return TN; }
+int attn_sm100_max_splits() { return 8; }
+
+// Key splits per row tile (the cluster size): the largest S <= 8 and <= the
+// tile count for which all `groups` clusters are resident in one wave; 1 if
+// even single CTAs need several waves.
+int attn_sm100_pick_splits(int D, long groups, int max_tiles) {
+    const int hi = max(1, min(8, max_tiles));
+    for (int S = hi; S > 1; --S) {
+        const int fit = D == 64 ? max_active_clusters<64>(S) : max_active_clusters<128>(S);
+        if (fit == 0 && S * groups <= kNumSMs) return S;  // query unavailable: assume one CTA per SM
+        if (fit >= groups) return S;
+    }
+    return 1;
+}
 
 cudaError_t attn_sm100_launch(const AttnParams &p, cudaStream_t s) {
     return p.D == 64 ? launch<64>(p, s) : launch<128>(p, s);

@@ -69,7 +69,8 @@ typedef enum {
 /* Attention                                                                 */
 /* ------------------------------------------------------------------------ */
 
-/* Bytes of workspace tidar_attn_step needs for these sizes (0 if invalid). */
+/* Bytes of workspace tidar_attn_step needs for these sizes (0 if invalid):
+ * the split-KV partial rows, which stay L2-resident. */
 size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max);
 
 /*
@@ -93,7 +94,7 @@ size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max
  * v_cache    bf16 [B, Hkv, P_max, D]
  * prefix_len int32 [B]  P_b, 0 <= P_b <= P_max
  * Hq % Hkv == 0; query head h reads KV head h / (Hq/Hkv).  D in {64, 128}.
- * softmax_scale  score multiplier (1/sqrt(D) for the standard scale).
+ * softmax_scale  score multiplier, > 0 (1/sqrt(D) for the standard scale).
  * out        bf16 [B, R, Hq, D]  softmax(scale * q k^T) v over the visible keys
  * lse        f32  [B, R, Hq] or NULL: natural-log log-sum-exp of the scaled scores
  * workspace  >= tidar_attn_workspace_size(...) bytes of device memory, 256-byte
