@@ -32,6 +32,7 @@ _SIGS = {
     "tidar_attn_step": (_i, [_vp] * 6 + [_i] * 6 + [_f, _i] + [_vp, _vp, _vp, _sz, _vp, _vp]),
     "tidar_verify_workspace_size": (_sz, [_i] * 3),
     "tidar_verify": (_i, [_vp, _vp, _i] + [_vp] * 4 + [_i] * 3 + [_vp] * 7 + [_sz, _vp, _vp]),
+    "tidar_verify_noalloc": (_i, [_vp, _vp, _i] + [_vp] * 4 + [_i] * 3 + [_vp] * 7 + [_vp]),
     "tidar_kv_commit_workspace_size": (_sz, [_i] * 3),
     "tidar_kv_commit": (_i, [_vp] * 4 + [_i] * 6 + [_vp] * 4 + [_i, _i, _vp] + [_vp] * 4 + [_sz, _vp, _vp]),
     "tidar_status_string": (ctypes.c_char_p, [_i]),
@@ -95,6 +96,16 @@ def tidar_verify(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u
         _ptr(p_logits), _ptr(q_logits), logits_dtype, _ptr(drafts), _ptr(preaccepted), _ptr(u_acc), _ptr(u_res),
         B, k, V, _ptr(accept_len), _ptr(resampled), _ptr(tokens), _ptr(n_emitted), _ptr(logp_d), _ptr(logq_d),
         _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def tidar_verify_noalloc(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u_res, B, k, V, accept_len,
+                         resampled, tokens, n_emitted, logp_d, logq_d, dev_status, stream=None) -> None:
+    """tidar_verify for callers that cannot allocate device memory: the scratch is a fixed 2 MiB array
+    inside the library, shared by every call on the device (overlapping calls race)."""
+    _check("tidar_verify_noalloc", _lib.tidar_verify_noalloc(
+        _ptr(p_logits), _ptr(q_logits), logits_dtype, _ptr(drafts), _ptr(preaccepted), _ptr(u_acc), _ptr(u_res),
+        B, k, V, _ptr(accept_len), _ptr(resampled), _ptr(tokens), _ptr(n_emitted), _ptr(logp_d), _ptr(logq_d),
+        _ptr(dev_status), _stream(stream)))
 
 
 def tidar_kv_commit_workspace_size(B, k, V) -> int:

@@ -149,6 +149,29 @@ tidar_status tidar_verify(const void *p_logits, const void *q_logits, int logits
                           float *logp_d, float *logq_d, void *workspace, size_t ws_bytes,
                           int32_t *dev_status, void *stream);
 
+/*
+ * tidar_verify without a caller workspace.  The paper has no counterpart: this
+ * entry point exists for callers that cannot allocate device memory -- e.g. a
+ * plug-in inside a host runtime that owns all device memory and forbids
+ * cudaMalloc on its decode path, or a serving loop that must not allocate after
+ * start-up -- and so cannot pass the workspace tidar_verify needs.
+ *
+ * Arguments, outputs, device-status bits and results are those of
+ * tidar_verify.  The scratch is a fixed 2 MiB device array inside the library
+ * (held by every GPU that loads it until the process exits); calls whose
+ * tidar_verify_workspace_size(B, k, V) exceeds 2 MiB return
+ * TIDAR_ERR_WORKSPACE without launching.  The first call on each device
+ * resolves the array's device address (cudaGetSymbolAddress) with that device
+ * current, so it should come before any stream capture.  All calls on a device
+ * share the array: calls whose kernels may overlap on the GPU race on it and
+ * must be ordered by the caller.  The library allocates nothing for this call.
+ */
+tidar_status tidar_verify_noalloc(const void *p_logits, const void *q_logits, int logits_dtype,
+                                  const int32_t *drafts, const uint8_t *preaccepted,
+                                  const float *u_acc, const float *u_res, int B, int k, int V,
+                                  int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
+                                  float *logp_d, float *logq_d, int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Commit                                                                    */
 /* ------------------------------------------------------------------------ */
