@@ -7,9 +7,11 @@
 // R new keys of this step in 128-row tiles.
 //
 // Warp roles (12 warps):
-//   warp 0      TMA producer: K and V tiles (128-byte swizzle) into a
-//               3-stage ring; prefix tiles from the cache, new-key tiles from
-//               K_new/V_new through a 3-D tensor map (no head gather).
+//   warps 0, 2  TMA producers of K and of V (128-byte swizzle), each into its
+//               own 3-stage ring: prefix tiles from the cache, new-key tiles
+//               from K_new/V_new through a 3-D tensor map (no head gather).
+//               A K stage is freed when its QK^T completes, a V stage when
+//               its PV does, so K runs ahead of V.
 //   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into the
 //               S columns of the warpgroup that owns the tile, then
 //               O += P V with P read from TMEM (tcgen05.mma A-from-TMEM).
@@ -20,7 +22,7 @@
 //               runs its exponentials.  The mask is evaluated from indices;
 //               O is rescaled only when the running max grows by more than
 //               2^8 (a stale max is exact as long as p <= 2^8 fits).
-//   warps 2-3   load Q when its rows cannot come through TMA, then idle.
+//   warps 2-3   also load Q when its rows cannot come through TMA.
 // TMEM (512 columns): warpgroup w owns S/P at [256w, 256w+128) and O at
 // [256w+128, 256w+128+D).  P (bf16) overwrites the first 64 columns of S; the
 // next S into those columns is issued after the PV that reads P, and
@@ -57,7 +59,7 @@ struct Smem {
     static constexpr int STAGE = 2 * KV_TILE;
     static constexpr int KV_OFF = Q_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
-    static constexpr int NBARS = 2 * STAGES + 7;  // kv_full, kv_empty, s_full[2], p_full[2], o_done[2], q_full
+    static constexpr int NBARS = 4 * STAGES + 7;  // k_full, k_empty, v_full, v_empty, s/p_full[2], o_done[2], q_full
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int ALLOC = TOTAL + 1024;  // alignment slack
@@ -69,6 +71,27 @@ __device__ __forceinline__ uint32_t range_bits(int a, int b, int base) {
     if (hi <= lo) return 0u;
     const uint32_t below_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
     return below_hi & ~((1u << lo) - 1u);
+}
+
+// S(tmem) = Q K^T: D/16 MMAs over the head dimension.  Q and K are K-major with 128-byte swizzle in
+// blocks of 64 columns (TM or TN rows x 128 B); within a block a 16-column step is +32 B (+2 in the
+// descriptor's address field).
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_s, uint64_t dq, uint64_t dk, uint32_t id) {
+    constexpr uint64_t kQBlock = (TM * 128) >> 4, kKBlock = (TN * 128) >> 4;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (kk & 3) * 2;
+        tc::mma_ss(d_s, dq + (kk >> 2) * kQBlock + off, dk + (kk >> 2) * kKBlock + off, id, kk > 0 ? 1u : 0u);
+    }
+}
+
+// O(tmem) (+)= P(tmem) V: TN/16 MMAs over the keys.  P occupies the first TN/2 columns of S (two bf16 per
+// column); V is MN-major, a 16-key step is 16 rows x 128 B (+128 in the descriptor's address field).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv, uint32_t id, bool acc) {
+#pragma unroll
+    for (int kk = 0; kk < TN / 16; ++kk) tc::mma_ts(d_o, a_p + kk * 8, dv + kk * 128, id, (acc || kk > 0) ? 1u : 0u);
 }
 
 // Number of valid keys in tile t (t < TP: prefix tile, else new-key tile).
@@ -88,12 +111,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t sQ = sbase;
     const uint32_t sKV = sbase + L::KV_OFF;
     const uint32_t bar0 = sbase + L::BAR_OFF;
-    auto kv_full = [&](int s) { return bar0 + 8u * s; };
-    auto kv_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
-    auto s_full = [&](int w) { return bar0 + 8u * (2 * STAGES + w); };
-    auto p_full = [&](int w) { return bar0 + 8u * (2 * STAGES + 2 + w); };
-    auto o_done = [&](int w) { return bar0 + 8u * (2 * STAGES + 4 + w); };
-    const uint32_t q_full = bar0 + 8u * (2 * STAGES + 6);
+    auto k_full = [&](int s) { return bar0 + 8u * s; };
+    auto k_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto v_full = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+    auto v_empty = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
+    auto s_full = [&](int w) { return bar0 + 8u * (4 * STAGES + w); };
+    auto p_full = [&](int w) { return bar0 + 8u * (4 * STAGES + 2 + w); };
+    auto o_done = [&](int w) { return bar0 + 8u * (4 * STAGES + 4 + w); };
+    const uint32_t q_full = bar0 + 8u * (4 * STAGES + 6);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -103,8 +128,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---- set-up that needs nothing from the previous kernel (programmatic dependent launch) ----
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            tc::mbar_init(kv_full(s), 1);
-            tc::mbar_init(kv_empty(s), 1);
+            tc::mbar_init(k_full(s), 1);
+            tc::mbar_init(k_empty(s), 1);
+            tc::mbar_init(v_full(s), 1);
+            tc::mbar_init(v_empty(s), 1);
         }
         for (int w = 0; w < 2; ++w) {
             tc::mbar_init(s_full(w), 1);
@@ -139,25 +166,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int t1 = (int)((long)(split + 1) * T / p.n_splits);
     const int n = t1 - t0;
 
-    auto issue_tile = [&](int i) {  // K and V of tile i into stage i % STAGES
+    // K (is_v = 0) or V (is_v = 1) of tile i into stage i % STAGES of its ring
+    auto issue_tile = [&](int i, int is_v) {
         const int st = i % STAGES;
-        tc::mbar_arrive_expect_tx(kv_full(st), L::STAGE);
+        const uint32_t bar = is_v ? v_full(st) : k_full(st);
+        tc::mbar_arrive_expect_tx(bar, L::KV_TILE);
         const int t = t0 + i;
-        const uint32_t kd = sKV + st * L::STAGE, vd = kd + L::KV_TILE;
+        const uint32_t dst = sKV + st * L::STAGE + is_v * L::KV_TILE;
         if (t < TP) {
             const int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) {
-                tc::tma_load_2d(kd + h * TN * 128, &tm_kc, h * 64, y, kv_full(st));
-                tc::tma_load_2d(vd + h * TN * 128, &tm_vc, h * 64, y, kv_full(st));
-            }
+            for (int h = 0; h < D / 64; ++h) tc::tma_load_2d(dst + h * TN * 128, is_v ? &tm_vc : &tm_kc, h * 64, y, bar);
         } else {
             const int z = b * p.R + (t - TP) * TN;
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) {
-                tc::tma_load_3d(kd + h * TN * 128, &tm_kn, h * 64, kvh, z, kv_full(st));
-                tc::tma_load_3d(vd + h * TN * 128, &tm_vn, h * 64, kvh, z, kv_full(st));
-            }
+            for (int h = 0; h < D / 64; ++h)
+                tc::tma_load_3d(dst + h * TN * 128, is_v ? &tm_vn : &tm_kn, h * 64, kvh, z, bar);
         }
     };
 
@@ -170,7 +194,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int h = 0; h < D / 64; ++h)
                 tc::tma_load_3d(sQ + h * TM * 128, &tm_q, h * 64, kvh * p.G, b * p.R + mt * (TM / p.G), q_full);
         }
-        for (int i = 0; i < prologue; ++i) issue_tile(i);
+        for (int i = 0; i < prologue; ++i) {
+            issue_tile(i, 0);
+            issue_tile(i, 1);
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -198,77 +225,79 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
-        if (warp == 0) {
-            // ================= TMA producer =================
+        if (warp == 0 || warp == 2) {
+            // ================= TMA producers: warp 0 streams K, warp 2 streams V =================
+            // K of a tile is released as soon as its QK^T completes, V after its PV, so the K ring
+            // runs ahead of the V ring and QK^T of the next tiles never waits behind a PV.
+            const int is_v = warp == 2;
             if (lane == 0) {
                 int issued = prologue;
                 for (int i = prologue; i < n; ++i) {
                     const int u = i / STAGES;
-                    if (!tc::mbar_wait(kv_empty(i % STAGES), (u - 1) & 1, abort_flag, kWaitCycles)) break;
-                    issue_tile(i);
+                    if (!tc::mbar_wait(is_v ? v_empty(i % STAGES) : k_empty(i % STAGES), (u - 1) & 1, abort_flag,
+                                       kWaitCycles))
+                        break;
+                    issue_tile(i, is_v);
                     issued = i + 1;
                 }
                 // drain: no copy may land after the CTA exits
                 for (int i = max(0, issued - STAGES); i < issued; ++i)
-                    tc::mbar_wait(kv_full(i % STAGES), (i / STAGES) & 1, abort_flag, kWaitCycles);
+                    tc::mbar_wait(is_v ? v_full(i % STAGES) : k_full(i % STAGES), (i / STAGES) & 1, abort_flag,
+                                  kWaitCycles);
             }
             __syncwarp();
         } else if (warp == 1) {
-            // ================= MMA issuer =================
+            // ================= MMA issuer (one thread issues, the warp waits) =================
+            // Order: QK(0), QK(1), then PV(i), QK(i+2) for every i -- QK(i+2) writes the S/P columns that
+            // PV(i) reads, and tcgen05.mma executes in issue order.
             constexpr uint32_t id_qk = tc::idesc_bf16_f32(TM, TN, 0, 0);
             constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
             bool ok = tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);
-            auto issue_qk = [&](int i) {
-                const int st = i % STAGES, w = i & 1;
-                ok = ok && tc::mbar_wait(kv_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
-                if (!ok) return;
-                const int valid = tile_valid(t0 + i, TP, P, p.R);
-                if (valid < TN) {  // keys past the sequence: zero their V rows so that 0 * V stays 0
-                    uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
-                    for (int idx = lane; idx < (TN - valid) * (D / 8); idx += 32) {
-                        const int j = valid + idx / (D / 8), c = idx % (D / 8);
-                        *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
-                            make_uint4(0, 0, 0, 0);
+            // descriptors are built once; a k-step or stage moves the start address, which lives in the low
+            // 14 bits (address >> 4; shared memory is < 256 KB, so the add never carries out)
+            const uint64_t dq = tc::smem_desc_sw128(sQ, 16, 1024);
+            const uint64_t dk = tc::smem_desc_sw128(sKV, 16, 1024);
+            const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
+            const uint32_t tb = tbase;
+            for (int it = 0; it < n + 2 && ok; ++it) {
+                if (it >= 2) {  // PV(i), i = it - 2
+                    const int i = it - 2, st = i % STAGES, w = i & 1;
+                    ok = tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
+                    if (!ok) break;
+                    const int valid = tile_valid(t0 + i, TP, P, p.R);
+                    if (valid < TN) {  // keys past the sequence: zero their V rows so that 0 * V stays 0
+                        uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
+                        for (int idx = lane; idx < (TN - valid) * (D / 8); idx += 32) {
+                            const int j = valid + idx / (D / 8), c = idx % (D / 8);
+                            *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                        tc::fence_proxy_async_smem();
                     }
-                    tc::fence_proxy_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    tc::fence_after_sync();
-                    const uint32_t kb = sKV + st * L::STAGE;
-    #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
-                        const uint64_t ad = tc::smem_desc_sw128(sQ + (kk >> 2) * TM * 128 + off, 16, 1024);
-                        const uint64_t bd = tc::smem_desc_sw128(kb + (kk >> 2) * TN * 128 + off, 16, 1024);
-                        tc::mma_ss(tbase + w * 256, ad, bd, id_qk, kk > 0);
+                    __syncwarp();
+                    ok = tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
+                    if (!ok) break;
+                    if (lane == 0) {
+                        tc::fence_after_sync();
+                        issue_pv<D>(tb + w * 256 + 128, tb + w * 256, dv + st * (uint64_t)(L::STAGE >> 4), id_pv,
+                                    i >= 2);
+                        tc::mma_commit(v_empty(st));
+                        if (i + 2 >= n) tc::mma_commit(o_done(w));
                     }
-                    tc::mma_commit(s_full(w));
+                    __syncwarp();
                 }
-                __syncwarp();
-            };
-            auto issue_pv = [&](int i) {
-                const int st = i % STAGES, w = i & 1;
-                ok = ok && tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
-                if (!ok) return;
-                if (lane == 0) {
-                    tc::fence_after_sync();
-                    const uint32_t vb = sKV + st * L::STAGE + L::KV_TILE;
-    #pragma unroll
-                    for (int kk = 0; kk < TN / 16; ++kk) {
-                        const uint64_t bd = tc::smem_desc_sw128(vb + kk * 16 * 128, TN * 128, 1024);
-                        tc::mma_ts(tbase + w * 256 + 128, tbase + w * 256 + kk * 8, bd, id_pv, (i >= 2 || kk > 0) ? 1u : 0u);
+                if (it < n) {  // QK(i), i = it
+                    const int i = it, st = i % STAGES, w = i & 1;
+                    ok = tc::mbar_wait(k_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
+                    if (!ok) break;
+                    if (lane == 0) {
+                        tc::fence_after_sync();
+                        issue_qk<D>(tb + w * 256, dq, dk + st * (uint64_t)(L::STAGE >> 4), id_qk);
+                        tc::mma_commit(s_full(w));
+                        tc::mma_commit(k_empty(st));
                     }
-                    tc::mma_commit(kv_empty(st));
-                    if (i + 2 >= n) tc::mma_commit(o_done(w));
+                    __syncwarp();
                 }
-                __syncwarp();
-            };
-            if (n > 0) issue_qk(0);
-            if (n > 1) issue_qk(1);
-            for (int i = 0; i < n && ok; ++i) {
-                issue_pv(i);
-                if (i + 2 < n) issue_qk(i + 2);
             }
         }
         __syncwarp();
@@ -465,9 +494,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
         const size_t group = (size_t)bh * (p.Mpad / TM) + mt;
         uint8_t *gbase = reinterpret_cast<uint8_t *>(p.part) + group * S * TM * REC;  // [S][TM][REC]
-        for (int idx = tid - 128; idx < TM * REC / 16; idx += 256)
-            reinterpret_cast<uint4 *>(gbase + (size_t)split * TM * REC)[idx] = reinterpret_cast<const uint4 *>(rec)[idx];
-        __threadfence();
+        if (S > 1) {  // the other CTAs of the cluster read these records; this CTA reads its own from smem
+            for (int idx = tid - 128; idx < TM * REC / 16; idx += 256)
+                reinterpret_cast<uint4 *>(gbase + (size_t)split * TM * REC)[idx] =
+                    reinterpret_cast<const uint4 *>(rec)[idx];
+            __threadfence();
+        }
         tc::fence_before_sync();
         tc::cluster_sync();
 
@@ -488,14 +520,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int sp = 0; sp < 8; ++sp) {
                     lsev[j][sp] = -INFINITY;
                     if (sp < S && lr < nrows) {
-                        const uint8_t *r0 = gbase + ((size_t)sp * TM + row0 + lr) * REC;
-                        const float *hd = reinterpret_cast<const float *>(r0 + 2 * D);
-                        lsev[j][sp] = __ldcg(hd);
-                        scl[j][sp] = __ldcg(hd + 1 + half);
-                        if constexpr (PER == 4)
-                            raw[j][sp] = __ldcg(reinterpret_cast<const uint2 *>(r0 + lane * PER * 2));
-                        else
-                            raw[j][sp].x = __ldcg(reinterpret_cast<const unsigned int *>(r0 + lane * PER * 2));
+                        if (sp == split) {  // own records: still in shared memory
+                            const uint8_t *r0 = rec + (row0 + lr) * REC;
+                            const float *hd = reinterpret_cast<const float *>(r0 + 2 * D);
+                            lsev[j][sp] = hd[0];
+                            scl[j][sp] = hd[1 + half];
+                            if constexpr (PER == 4)
+                                raw[j][sp] = *reinterpret_cast<const uint2 *>(r0 + lane * PER * 2);
+                            else
+                                raw[j][sp].x = *reinterpret_cast<const unsigned int *>(r0 + lane * PER * 2);
+                        } else {
+                            const uint8_t *r0 = gbase + ((size_t)sp * TM + row0 + lr) * REC;
+                            const float *hd = reinterpret_cast<const float *>(r0 + 2 * D);
+                            lsev[j][sp] = __ldcg(hd);
+                            scl[j][sp] = __ldcg(hd + 1 + half);
+                            if constexpr (PER == 4)
+                                raw[j][sp] = __ldcg(reinterpret_cast<const uint2 *>(r0 + lane * PER * 2));
+                            else
+                                raw[j][sp].x = __ldcg(reinterpret_cast<const unsigned int *>(r0 + lane * PER * 2));
+                        }
                     }
                 }
             }

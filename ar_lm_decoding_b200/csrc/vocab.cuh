@@ -167,6 +167,89 @@ __device__ __forceinline__ int chunk_search(const double (&w)[8], double target,
     return pick[0] != 0x7fffffff ? pick[0] : pick[1];
 }
 
+// This thread's 32 consecutive entries (tid*32 .. tid*32+31) of chunk c (256 threads), -inf beyond V.
+__device__ __forceinline__ void load_chunk32_contig(const void *row, int dtype, int V, int c, float (&v)[32]) {
+    const int i0 = c * kChunk + threadIdx.x * 32;
+    if (dtype == TIDAR_DT_BF16) {
+        const bf16 *r = reinterpret_cast<const bf16 *>(row);
+        if (i0 + 32 <= V && ((reinterpret_cast<uintptr_t>(r + i0) & 15) == 0)) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(r + i0) + q);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    v[q * 8 + 2 * e] = __uint_as_float(w[e] << 16);
+                    v[q * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = i0 + e < V ? __bfloat162float(r[i0 + e]) : -INFINITY;
+        }
+    } else {
+        const float *r = reinterpret_cast<const float *>(row);
+        if (i0 + 32 <= V && ((reinterpret_cast<uintptr_t>(r + i0) & 15) == 0)) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(r + i0) + q);
+                v[q * 4 + 0] = a.x; v[q * 4 + 1] = a.y; v[q * 4 + 2] = a.z; v[q * 4 + 3] = a.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = i0 + e < V ? r[i0 + e] : -INFINITY;
+        }
+    }
+}
+
+// Ordered search inside one chunk with 256 threads holding 32 consecutive weights each (entries
+// tid*32 .. tid*32+31): the first local index whose inclusive sum exceeds `target`, or the last
+// index with positive weight when rounding leaves none (target beyond the chunk's total).
+__device__ __forceinline__ int chunk_search256(const double (&w)[32], double target, double *scan_buf, int *pick) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    double loc = 0.0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) loc += w[e];
+    double incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (tid == 0) { pick[0] = 0x7fffffff; pick[1] = -1; }
+    if (lane == 31) scan_buf[warp] = incl;
+    __syncthreads();
+    double before = 0.0;
+    for (int i = 0; i < warp; ++i) before += scan_buf[i];
+    double c = before + incl - loc;  // exclusive prefix of this thread
+    int first = 0x7fffffff, last = -1;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        c += w[e];
+        if (w[e] > 0.0) {
+            last = tid * 32 + e;
+            if (c > target && first == 0x7fffffff) first = tid * 32 + e;
+        }
+    }
+    if (first != 0x7fffffff) atomicMin(&pick[0], first);
+    if (last >= 0) atomicMax(&pick[1], last);
+    __syncthreads();
+    return pick[0] != 0x7fffffff ? pick[0] : pick[1];
+}
+
+// Merge of chunk statistics by up to 32 lanes of one warp (lane c takes chunk c, c + 32, ...):
+// every lane returns the row max m and the row sum Z of exp(x - m).
+__device__ __forceinline__ void merge_stats_warp(const ChunkStat *st, int n, float &m, double &z) {
+    const int lane = threadIdx.x & 31;
+    float mx = -INFINITY;
+    for (int c = lane; c < n; c += 32) mx = fmaxf(mx, st[c].m);
+    m = warp_max(mx);
+    double s = 0.0;
+    for (int c = lane; c < n; c += 32)
+        if (st[c].m != -INFINITY) s += st[c].z * (double)exp2f((st[c].m - m) * kLog2e);
+    z = warp_sum_d(s);
+}
+
 // This thread's 8 consecutive entries (tid*8..tid*8+7) of chunk c as floats (-inf beyond V).
 __device__ __forceinline__ void load_chunk8(const void *row, int dtype, int V, int c, float (&v)[8]) {
     const int i0 = c * kChunk + threadIdx.x * 8;

@@ -260,8 +260,9 @@ def gpu_smi_id(device):
 
 
 def kernels_per_step(cfg):
-    # per layer: one attention kernel (split-KV merged in-kernel); verify: 3; commit: 2
-    return cfg.L + 3 + 2
+    # per layer: one attention kernel (split-KV merged in-kernel); verify: 2 (vocab statistics, decision);
+    # commit: 1 (its counters are zeroed by a memset node, not a kernel)
+    return cfg.L + 2 + 1
 
 
 def gpu_arm(args, cfg):
