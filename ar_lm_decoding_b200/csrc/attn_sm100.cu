@@ -50,6 +50,7 @@ constexpr int TM = 128;
 constexpr int TN = 128;
 constexpr int STAGES = 3;
 constexpr int THREADS = 384;
+constexpr int kMaxSplits = 8;  // cluster size limit (portable clusters)
 constexpr long long kWaitCycles = 4000000000LL;
 
 template <int D>
@@ -92,6 +93,74 @@ template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv, uint32_t id, bool acc) {
 #pragma unroll
     for (int kk = 0; kk < TN / 16; ++kk) tc::mma_ts(d_o, a_p + kk * 8, dv + kk * 128, id, (acc || kk > 0) ? 1u : 0u);
+}
+
+// Row maximum of the raw scores of one S tile (this thread's TMEM lane, TN columns).  MASKED: only keys
+// in [0, lo) and [glo, ghi) count.
+template <bool MASKED>
+__device__ __forceinline__ float tile_max(uint32_t s_col, int lo, int glo, int ghi) {
+    float x[TN];
+#pragma unroll
+    for (int c = 0; c < TN / 32; ++c) {
+        uint32_t v[32];
+        tc::tmem_ld32(s_col + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[c * 32 + j] = __uint_as_float(v[j]);
+    }
+    tc::tmem_wait_ld();
+    if constexpr (MASKED) {
+#pragma unroll
+        for (int c = 0; c < TN / 32; ++c) {
+            const uint32_t bits = range_bits(0, lo, c * 32) | range_bits(glo, ghi, c * 32);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[c * 32 + j] = (bits >> j) & 1u ? x[c * 32 + j] : -INFINITY;
+        }
+    }
+    float m8[8];  // eight independent chains
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m8[j] = x[j];
+#pragma unroll
+    for (int j = 8; j < TN; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+    return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
+// p = 2^(s * sl2 + neg_m) for one S tile, written back over S as bf16 pairs (P, the A operand of PV), in
+// 64-column chunks that re-read S from TMEM (a rolled loop keeps the code small).  Returns the row sum
+// of p.  Chunk c writes TMEM columns [32c, 32c + 32), which chunks > c do not read.
+template <bool MASKED>
+__device__ __forceinline__ float tile_exp(uint32_t s_col, int lo, int glo, int ghi, float sl2, float neg_m) {
+    float sum8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < TN / 64; ++c) {
+        uint32_t v0[32], v1[32];
+        tc::tmem_ld32(s_col + c * 64, v0);
+        tc::tmem_ld32(s_col + c * 64 + 32, v1);
+        tc::tmem_wait_ld();
+        uint32_t bits0 = 0xffffffffu, bits1 = 0xffffffffu;
+        if constexpr (MASKED) {
+            bits0 = range_bits(0, lo, c * 64) | range_bits(glo, ghi, c * 64);
+            bits1 = range_bits(0, lo, c * 64 + 32) | range_bits(glo, ghi, c * 64 + 32);
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const uint32_t *v = j < 16 ? v0 : v1;
+            float a = fast_exp2(fmaf(__uint_as_float(v[(2 * j) & 31]), sl2, neg_m));
+            float bb = fast_exp2(fmaf(__uint_as_float(v[(2 * j + 1) & 31]), sl2, neg_m));
+            if constexpr (MASKED) {
+                const uint32_t bits = j < 16 ? bits0 : bits1;
+                a = (bits >> ((2 * j) & 31)) & 1u ? a : 0.f;
+                bb = (bits >> ((2 * j + 1) & 31)) & 1u ? bb : 0.f;
+            }
+            sum8[(2 * j) & 7] += a;
+            sum8[(2 * j + 1) & 7] += bb;
+            pk[j] = pack_bf16x2(a, bb);
+        }
+        tc::tmem_st32(s_col + c * 32, pk);
+    }
+    return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 }
 
 // Number of valid keys in tile t (t < TP: prefix tile, else new-key tile).
@@ -247,56 +316,51 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             __syncwarp();
         } else if (warp == 1) {
-            // ================= MMA issuer (one thread issues, the warp waits) =================
+            // ================= MMA issuer: one thread runs the whole loop =================
             // Order: QK(0), QK(1), then PV(i), QK(i+2) for every i -- QK(i+2) writes the S/P columns that
-            // PV(i) reads, and tcgen05.mma executes in issue order.
-            constexpr uint32_t id_qk = tc::idesc_bf16_f32(TM, TN, 0, 0);
-            constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
-            bool ok = tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);
-            // descriptors are built once; a k-step or stage moves the start address, which lives in the low
-            // 14 bits (address >> 4; shared memory is < 256 KB, so the add never carries out)
-            const uint64_t dq = tc::smem_desc_sw128(sQ, 16, 1024);
-            const uint64_t dk = tc::smem_desc_sw128(sKV, 16, 1024);
-            const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
-            const uint32_t tb = tbase;
-            for (int it = 0; it < n + 2 && ok; ++it) {
-                if (it >= 2) {  // PV(i), i = it - 2
-                    const int i = it - 2, st = i % STAGES, w = i & 1;
-                    ok = tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
-                    if (!ok) break;
-                    const int valid = tile_valid(t0 + i, TP, P, p.R);
-                    if (valid < TN) {  // keys past the sequence: zero their V rows so that 0 * V stays 0
-                        uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
-                        for (int idx = lane; idx < (TN - valid) * (D / 8); idx += 32) {
-                            const int j = valid + idx / (D / 8), c = idx % (D / 8);
-                            *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
-                                make_uint4(0, 0, 0, 0);
-                        }
-                        tc::fence_proxy_async_smem();
-                    }
-                    __syncwarp();
-                    ok = tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
-                    if (!ok) break;
-                    if (lane == 0) {
+            // PV(i) reads, and tcgen05.mma executes in issue order.  The loop has no warp-wide operation and
+            // no division: its thread spends its time in barrier waits and MMA issue.
+            if (lane == 0) {
+                constexpr uint32_t id_qk = tc::idesc_bf16_f32(TM, TN, 0, 0);
+                constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
+                constexpr uint64_t kStage = L::STAGE >> 4;  // one ring stage in the descriptor's address field
+                // descriptors are built once; a k-step or stage moves the start address, which lives in the
+                // low 14 bits (address >> 4; shared memory is < 256 KB, so the add never carries out)
+                const uint64_t dq = tc::smem_desc_sw128(sQ, 16, 1024);
+                const uint64_t dk = tc::smem_desc_sw128(sKV, 16, 1024);
+                const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
+                const uint32_t tb = tbase;
+                bool ok = tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);
+                int kst = 0, vst = 0;       // ring stages of the next QK and the next PV
+                uint32_t kph = 0, vph = 0;  // and the phase parities they wait for
+                for (int it = 0; ok && it < n + 2; ++it) {
+                    if (it >= 2) {  // PV(i), i = it - 2
+                        const int i = it - 2, w = i & 1;
+                        ok = tc::mbar_wait(v_full(vst), vph, abort_flag, kWaitCycles) &&
+                             tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
+                        if (!ok) break;
                         tc::fence_after_sync();
-                        issue_pv<D>(tb + w * 256 + 128, tb + w * 256, dv + st * (uint64_t)(L::STAGE >> 4), id_pv,
-                                    i >= 2);
-                        tc::mma_commit(v_empty(st));
+                        issue_pv<D>(tb + w * 256 + 128, tb + w * 256, dv + vst * kStage, id_pv, i >= 2);
+                        tc::mma_commit(v_empty(vst));
                         if (i + 2 >= n) tc::mma_commit(o_done(w));
+                        if (++vst == STAGES) {
+                            vst = 0;
+                            vph ^= 1u;
+                        }
                     }
-                    __syncwarp();
-                }
-                if (it < n) {  // QK(i), i = it
-                    const int i = it, st = i % STAGES, w = i & 1;
-                    ok = tc::mbar_wait(k_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles);
-                    if (!ok) break;
-                    if (lane == 0) {
+                    if (it < n) {  // QK(it)
+                        const int w = it & 1;
+                        ok = tc::mbar_wait(k_full(kst), kph, abort_flag, kWaitCycles);
+                        if (!ok) break;
                         tc::fence_after_sync();
-                        issue_qk<D>(tb + w * 256, dq, dk + st * (uint64_t)(L::STAGE >> 4), id_qk);
+                        issue_qk<D>(tb + w * 256, dq, dk + kst * kStage, id_qk);
                         tc::mma_commit(s_full(w));
-                        tc::mma_commit(k_empty(st));
+                        tc::mma_commit(k_empty(kst));
+                        if (++kst == STAGES) {
+                            kst = 0;
+                            kph ^= 1u;
+                        }
                     }
-                    __syncwarp();
                 }
             }
         }
@@ -333,23 +397,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = w; i < n; i += 2) {
             if (!tc::mbar_wait(s_full(w), (i >> 1) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
             tc::fence_after_sync();
-            float x[TN];
-#pragma unroll
-            for (int c = 0; c < TN / 32; ++c) {
-                uint32_t v[32];
-                tc::tmem_ld32(s_col + c * 32, v);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[c * 32 + j] = __uint_as_float(v[j]);
-            }
-            tc::tmem_wait_ld();
             const int t = t0 + i;
-            if (t >= TP - 1 && !(t == TP - 1 && P % TN == 0)) {
-                // partial prefix tile (keys beyond P) or new-key tile (the TiDAR mask): visible keys of this
-                // row are [0, lo) and [glo, ghi), all below `end`
-                int lo, glo, ghi, end;
+            // a partial prefix tile (keys beyond P) or a new-key tile (the TiDAR mask): the visible keys of
+            // this row are [0, lo) and [glo, ghi); everything else, garbage included, is excluded by select
+            const bool masked = t >= TP - 1 && !(t == TP - 1 && P % TN == 0);
+            int lo = TN, glo = 0, ghi = 0;
+            if (masked) {
+                int end;
                 if (t < TP) {
                     lo = end = P - t * TN;
-                    glo = ghi = 0;
                 } else {
                     const int nn0 = (t - TP) * TN;
                     lo = vis_lim - nn0;
@@ -359,25 +415,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 lo = min(lo, end);
                 ghi = min(ghi, end);
-#pragma unroll
-                for (int c = 0; c < TN / 32; ++c) {
-                    const uint32_t bits = range_bits(0, lo, c * 32) | range_bits(glo, ghi, c * 32);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) x[c * 32 + j] = (bits >> j) & 1u ? x[c * 32 + j] : -INFINITY;
-                }
             }
-            float mx8[8];  // eight independent chains
-#pragma unroll
-            for (int j = 0; j < 8; ++j) mx8[j] = x[j];
-#pragma unroll
-            for (int j = 8; j < TN; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], x[j]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+            const float mx = (masked ? tile_max<true>(s_col, lo, glo, ghi) : tile_max<false>(s_col, lo, glo, ghi)) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + 8.f;
             if (i >= 2 && __any_sync(0xffffffffu, grow)) {  // rescale O (last written by the PV of tile i-2)
                 const float f = grow ? fast_exp2(m_run - m_new) : 1.f;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
                     tc::tmem_ld32(o_col + c * 32, v);
@@ -392,196 +436,147 @@ __global__ void __launch_bounds__(THREADS, 1)
                 m_run = m_new;
             }
             const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-            float sum8[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
-#pragma unroll
-            for (int c = 0; c < TN / 64; ++c) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float a = fast_exp2(fmaf(x[c * 64 + 2 * j], sl2, neg_m));
-                    const float bb = fast_exp2(fmaf(x[c * 64 + 2 * j + 1], sl2, neg_m));
-                    sum8[(2 * j) & 7] += a;
-                    sum8[(2 * j + 1) & 7] += bb;
-                    pk[j] = pack_bf16x2(a, bb);
+            l_run += masked ? tile_exp<true>(s_col, lo, glo, ghi, sl2, neg_m) : tile_exp<false>(s_col, lo, glo, ghi, sl2, neg_m);
+            const int valid = tile_valid(t, TP, P, p.R);
+            if (valid < TN) {
+                // keys past the sequence: zero their V rows (0 * garbage could be NaN) before PV reads them
+                const int st = i % STAGES;
+                if (!tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
+                uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
+                for (int idx = row; idx < (TN - valid) * (D / 8); idx += 128) {
+                    const int j = valid + idx / (D / 8), c = idx % (D / 8);
+                    *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
+                        make_uint4(0, 0, 0, 0);
                 }
-                tc::tmem_st32(s_col + c * 32, pk);
+                tc::fence_proxy_async_smem();
             }
-            l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(p_full(w));
         }
         // the next kernel in the stream may launch now: it waits for this grid before touching memory
         asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-        // ---- merge the two warpgroups (each takes half the columns), then one partial row per CTA ----
-        const bool has = n > w;
-        if (ok && has) ok = tc::mbar_wait(o_done(w), 0, abort_flag, kWaitCycles);
+        // ---- merge the two warpgroups' states.  A thread may read every TMEM column of its lane quadrant, so
+        // warpgroup w combines columns [w*D/2, (w+1)*D/2) of BOTH O accumulators straight from TMEM; only the
+        // row statistics (m, l) pass through shared memory ----
+        constexpr int H = D / 2;
+        for (int v = 0; v < 2 && ok; ++v)  // both accumulators final (the ring is idle from here on)
+            if (n > v) ok = tc::mbar_wait(o_done(v), 0, abort_flag, kWaitCycles);
         tc::fence_after_sync();
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");  // both warpgroups' MMAs done: the ring is free
-        constexpr int H = D / 2;     // columns merged by one warpgroup
-        constexpr int HS = H + 4;    // exchange row stride (floats)
-        constexpr int REC = 2 * D + 16;  // partial record: D fp16 values, then lse2, scale[2], pad (bytes)
-        float *xh = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM][HS]: the half the other WG merges
-        float *xml = xh + 2 * TM * HS;                              // [2][2][TM]: m, l
-        uint8_t *rec = reinterpret_cast<uint8_t *>(xml + 4 * TM);   // [TM][REC]
-        const int other = 1 - w;
-        const float m_self = has ? m_run : -INFINITY, l_self = has ? l_run : 0.f;
-#pragma unroll
-        for (int c = 0; c < H / 32; ++c) {
-            uint32_t v[32];
-            if (has && ok) {
-                tc::tmem_ld32(o_col + other * H + c * 32, v);
-                tc::tmem_wait_ld();
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = 0u;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4 *>(xh + (w * TM + row) * HS + c * 32 + j) =
-                    make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                __uint_as_float(v[j + 3]));
-        }
-        xml[(w * 2 + 0) * TM + row] = m_self;
-        xml[(w * 2 + 1) * TM + row] = l_self;
+        float *xml = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][2][TM]: m, l of each warpgroup
+        xml[(w * 2 + 0) * TM + row] = n > w ? m_run : -INFINITY;
+        xml[(w * 2 + 1) * TM + row] = n > w ? l_run : 0.f;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        const float m_o = xml[(other * 2 + 0) * TM + row], l_o = xml[(other * 2 + 1) * TM + row];
-        const float mm = fmaxf(m_self, m_o);
-        const float a_s = m_self == -INFINITY ? 0.f : fast_exp2(m_self - mm);
-        const float a_o = m_o == -INFINITY ? 0.f : fast_exp2(m_o - mm);
-        const float lt = l_self * a_s + l_o * a_o;
+        const float m0 = xml[row], l0 = xml[TM + row], m1 = xml[2 * TM + row], l1 = xml[3 * TM + row];
+        const float mm = fmaxf(m0, m1);
+        const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
+        const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
+        const float lt = l0 * a0 + l1 * a1;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float f_s = (has && ok) ? a_s * inv : 0.f, f_o = a_o * inv;
+        const float lse2 = lt > 0.f ? mm + __log2f(lt) : -INFINITY;  // log2 of this CTA's row sum
+        // tcgen05.ld is warp-collective: the decision to read an accumulator must be warp-uniform
+        const bool rd0 = __all_sync(0xffffffffu, ok && n > 0), rd1 = __all_sync(0xffffffffu, ok && n > 1);
+        const float f0 = rd0 ? a0 * inv : 0.f, f1 = rd1 ? a1 * inv : 0.f;
+        const uint32_t o0 = tbase + lane_off + 128 + w * H, o1 = tbase + lane_off + 256 + 128 + w * H;
         float hv[H];
 #pragma unroll
         for (int c = 0; c < H / 32; ++c) {
-            uint32_t v[32];
-            if (has && ok) {
-                tc::tmem_ld32(o_col + w * H + c * 32, v);
-                tc::tmem_wait_ld();
-            } else {
+            uint32_t v0[32], v1[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = 0u;
-            }
+            for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0u;
+            if (rd0) tc::tmem_ld32(o0 + c * 32, v0);
+            if (rd1) tc::tmem_ld32(o1 + c * 32, v1);
+            tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                hv[c * 32 + j] = __uint_as_float(v[j]) * f_s + xh[(other * TM + row) * HS + c * 32 + j] * f_o;
+            for (int j = 0; j < 32; ++j) hv[c * 32 + j] = __uint_as_float(v0[j]) * f0 + __uint_as_float(v1[j]) * f1;
         }
-        float amax = 0.f;
-#pragma unroll
-        for (int j = 0; j < H; ++j) amax = fmaxf(amax, fabsf(hv[j]));
-        const float scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
-        const float rs = 1.f / scale;
-        uint8_t *myrec = rec + row * REC;
-#pragma unroll
-        for (int j = 0; j < H; j += 8) {
-            uint4 u;
-            u.x = pack_half2(hv[j] * rs, hv[j + 1] * rs);
-            u.y = pack_half2(hv[j + 2] * rs, hv[j + 3] * rs);
-            u.z = pack_half2(hv[j + 4] * rs, hv[j + 5] * rs);
-            u.w = pack_half2(hv[j + 6] * rs, hv[j + 7] * rs);
-            *reinterpret_cast<uint4 *>(myrec + (w * H + j) * 2) = u;
-        }
-        float *hdr = reinterpret_cast<float *>(myrec + 2 * D);
-        hdr[1 + w] = scale;
-        if (w == 0) {
-            hdr[0] = lt > 0.f ? mm + __log2f(lt) : -INFINITY;
-            hdr[3] = 0.f;
-        }
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");
         const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
         const size_t group = (size_t)bh * (p.Mpad / TM) + mt;
-        uint8_t *gbase = reinterpret_cast<uint8_t *>(p.part) + group * S * TM * REC;  // [S][TM][REC]
-        if (S > 1) {  // the other CTAs of the cluster read these records; this CTA reads its own from smem
-            for (int idx = tid - 128; idx < TM * REC / 16; idx += 256)
-                reinterpret_cast<uint4 *>(gbase + (size_t)split * TM * REC)[idx] =
-                    reinterpret_cast<const uint4 *>(rec)[idx];
-            __threadfence();
+        // partial records of the row tile: vals [S][D/8][TM] (16 B = 8 fp16 per chunk: a warp's stores are
+        // contiguous), then hdr [S][TM] float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), 0)
+        uint8_t *gbase = reinterpret_cast<uint8_t *>(p.part) + group * S * TM * (2 * D + 16);
+        uint4 *vals = reinterpret_cast<uint4 *>(gbase);
+        float4 *hdr = reinterpret_cast<float4 *>(gbase + (size_t)S * TM * 2 * D);
+        if (S == 1) {  // the CTA saw every key of its rows: normalised output straight from the merge
+            if (m_row < p.M) {
+                const size_t orow = (size_t)(b * p.R + r) * p.Hq + kvh * p.G + (m_row - r * p.G);
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + w * H);
+#pragma unroll
+                for (int j = 0; j < H / 8; ++j)
+                    dst[j] = make_uint4(pack_bf16x2(hv[8 * j], hv[8 * j + 1]), pack_bf16x2(hv[8 * j + 2], hv[8 * j + 3]),
+                                        pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
+                if (w == 0 && p.lse) p.lse[orow] = lse2 * kLn2;
+            }
+        } else {
+            float amax = 0.f;
+#pragma unroll
+            for (int j = 0; j < H; ++j) amax = fmaxf(amax, fabsf(hv[j]));
+            const float scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
+            const float rs = 1.f / scale;
+            uint4 *vrec = vals + ((size_t)split * (D / 8) + w * (H / 8)) * TM + row;
+#pragma unroll
+            for (int j = 0; j < H / 8; ++j)
+                vrec[(size_t)j * TM] =
+                    make_uint4(pack_half2(hv[8 * j] * rs, hv[8 * j + 1] * rs), pack_half2(hv[8 * j + 2] * rs, hv[8 * j + 3] * rs),
+                               pack_half2(hv[8 * j + 4] * rs, hv[8 * j + 5] * rs), pack_half2(hv[8 * j + 6] * rs, hv[8 * j + 7] * rs));
+            float *h = reinterpret_cast<float *>(hdr + (size_t)split * TM + row);
+            h[1 + w] = scale;
+            if (w == 0) {
+                h[0] = lse2;
+                h[3] = 0.f;
+            }
         }
+        // the records reach the other CTAs of the cluster through the barrier's release / acquire
         tc::fence_before_sync();
         tc::cluster_sync();
 
-        // ---- merge the S partials of this CTA's slice of rows (L2-resident) ----
-        const int per = ceil_div(TM, S);
-        const int row0 = split * per, nrows = min(TM, row0 + per) - row0;
-        const int wi = warp - 4;  // 8 merging warps
-        constexpr int PER = D / 32;  // columns per lane
-        const int half = (lane * PER) / H;
-        // a warp takes rows wi, wi+8, ...; two at a time with all their records (<= 2 x 8) in flight
-        for (int lr0 = wi; lr0 < nrows; lr0 += 16) {
-            float lsev[2][8], scl[2][8];
-            uint2 raw[2][8];
+        if (S > 1) {
+            // ---- merge this CTA's slice of rows over the cluster's S partial records (L2-resident) ----
+            // item = (16-byte column chunk c, row): consecutive threads take consecutive rows of one chunk, so
+            // every load below is coalesced; each thread issues all of an item's loads before using any
+            const int per = ceil_div(TM, S);
+            const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
+            for (int it = tid - 128; it < nrows * (D / 8); it += 256) {
+                const int c = it / nrows, rr = row0 + (it - c * nrows);
+                float l2v[kMaxSplits], sc[kMaxSplits];
+                uint4 raw[kMaxSplits];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int lr = lr0 + 8 * j;
-#pragma unroll
-                for (int sp = 0; sp < 8; ++sp) {
-                    lsev[j][sp] = -INFINITY;
-                    if (sp < S && lr < nrows) {
-                        if (sp == split) {  // own records: still in shared memory
-                            const uint8_t *r0 = rec + (row0 + lr) * REC;
-                            const float *hd = reinterpret_cast<const float *>(r0 + 2 * D);
-                            lsev[j][sp] = hd[0];
-                            scl[j][sp] = hd[1 + half];
-                            if constexpr (PER == 4)
-                                raw[j][sp] = *reinterpret_cast<const uint2 *>(r0 + lane * PER * 2);
-                            else
-                                raw[j][sp].x = *reinterpret_cast<const unsigned int *>(r0 + lane * PER * 2);
-                        } else {
-                            const uint8_t *r0 = gbase + ((size_t)sp * TM + row0 + lr) * REC;
-                            const float *hd = reinterpret_cast<const float *>(r0 + 2 * D);
-                            lsev[j][sp] = __ldcg(hd);
-                            scl[j][sp] = __ldcg(hd + 1 + half);
-                            if constexpr (PER == 4)
-                                raw[j][sp] = __ldcg(reinterpret_cast<const uint2 *>(r0 + lane * PER * 2));
-                            else
-                                raw[j][sp].x = __ldcg(reinterpret_cast<const unsigned int *>(r0 + lane * PER * 2));
-                        }
-                    }
+                for (int sp = 0; sp < kMaxSplits; ++sp) {  // unconditional loads (clamped index), masked below
+                    const int sq = min(sp, S - 1);
+                    const float4 hd = __ldcg(hdr + (size_t)sq * TM + rr);
+                    raw[sp] = __ldcg(vals + ((size_t)sq * (D / 8) + c) * TM + rr);
+                    l2v[sp] = sp < S ? hd.x : -INFINITY;
+                    sc[sp] = c < D / 16 ? hd.y : hd.z;
                 }
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int lr = lr0 + 8 * j;
-                const int m = mt * TM + row0 + lr;
-                if (lr >= nrows || m >= p.M) continue;
                 float mx = -INFINITY;
 #pragma unroll
-                for (int sp = 0; sp < 8; ++sp) mx = fmaxf(mx, lsev[j][sp]);
-                float acc[PER], wsum = 0.f;
+                for (int sp = 0; sp < kMaxSplits; ++sp) mx = fmaxf(mx, l2v[sp]);
+                float acc[8], wsum = 0.f;
 #pragma unroll
-                for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+                for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-                for (int sp = 0; sp < 8; ++sp) {
-                    if (lsev[j][sp] != -INFINITY) {
-                        const float wq = fast_exp2(lsev[j][sp] - mx);
-                        wsum += wq;
-                        const float f = wq * scl[j][sp];
-                        const float2 v0 = unpack_half2(raw[j][sp].x);
-                        acc[0] += f * v0.x;
-                        acc[1] += f * v0.y;
-                        if constexpr (PER == 4) {
-                            const float2 v1 = unpack_half2(raw[j][sp].y);
-                            acc[2] += f * v1.x;
-                            acc[3] += f * v1.y;
-                        }
+                for (int sp = 0; sp < kMaxSplits; ++sp) {
+                    const float wq = l2v[sp] == -INFINITY ? 0.f : fast_exp2(l2v[sp] - mx);
+                    wsum += wq;
+                    const float f = wq * sc[sp];
+                    const uint32_t u[4] = {raw[sp].x, raw[sp].y, raw[sp].z, raw[sp].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v = unpack_half2(u[e]);
+                        acc[2 * e] += f * v.x;
+                        acc[2 * e + 1] += f * v.y;
                     }
                 }
-                const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
-                const int rq = m / p.G, h = kvh * p.G + (m - rq * p.G);
-                const size_t orow = (size_t)(b * p.R + rq) * p.Hq + h;
-                bf16 *dst = p.out + orow * D + lane * PER;
-                if constexpr (PER == 4) {
-                    uint2 v;
-                    v.x = pack_bf16x2(acc[0] * winv, acc[1] * winv);
-                    v.y = pack_bf16x2(acc[2] * winv, acc[3] * winv);
-                    *reinterpret_cast<uint2 *>(dst) = v;
-                } else {
-                    *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * winv, acc[1] * winv);
+                const int m = mt * TM + rr;
+                if (m < p.M) {
+                    const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+                    const int rq = m / p.G;
+                    const size_t orow = (size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G);
+                    *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) =
+                        make_uint4(pack_bf16x2(acc[0] * winv, acc[1] * winv), pack_bf16x2(acc[2] * winv, acc[3] * winv),
+                                   pack_bf16x2(acc[4] * winv, acc[5] * winv), pack_bf16x2(acc[6] * winv, acc[7] * winv));
+                    if (c == 0 && p.lse) p.lse[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
                 }
-                if (p.lse && lane == 0) p.lse[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
             }
         }
     }
@@ -689,7 +684,7 @@ int max_active_clusters(int S) {
 
 int attn_sm100_rows_per_tile() { return TM; }
 int attn_sm100_keys_per_tile() { return TN; }
-int attn_sm100_max_splits() { return 8; }
+int attn_sm100_max_splits() { return kMaxSplits; }
 
 // Key splits per row tile (the cluster size): the largest S <= 8 and <= the
 // tile count for which all `groups` clusters are resident in one wave; 1 if
