@@ -41,8 +41,7 @@ AttnPlan plan_attn(int B, int Hq, int Hkv, int D, int k, int P_max) {
     pl.mtiles = mtiles;
     pl.max_tiles = ceil_div(P_max, keys) + ceil_div(pl.R, keys);
     pl.n_splits = 0;  // chosen at launch (needs the device's cluster occupancy)
-    // one partial-row record (D fp16 + 16 bytes) per row of every split, sized for the largest cluster
-    pl.ws_bytes = align256((size_t)B * Hkv * mtiles * attn_sm100_max_splits() * rows * (2 * D + 16));
+    pl.ws_bytes = 0;  // split-KV partials move through the cluster's distributed shared memory
     pl.status = TIDAR_OK;
     return pl;
 }
@@ -67,15 +66,17 @@ tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new
                              size_t ws_bytes, int32_t *dev_status, void *stream) {
     const AttnPlan pl = plan_attn(B, Hq, Hkv, D, k, P_max);
     if (pl.status != TIDAR_OK) return pl.status;
-    if (!q || !k_new || !v_new || !k_cache || !v_cache || !prefix_len || !out || !dev_status || !workspace)
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !prefix_len || !out || !dev_status)
         return TIDAR_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
         !aligned16(out) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
         return TIDAR_ERR_INVALID_ARG;
     if (mask_mode != TIDAR_MASK_HYBRID && mask_mode != TIDAR_MASK_CAUSAL) return TIDAR_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.f)) return TIDAR_ERR_INVALID_ARG;
-    if (!aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
-    if (ws_bytes < pl.ws_bytes) return TIDAR_ERR_WORKSPACE;
+    if (pl.ws_bytes > 0) {
+        if (!workspace || !aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
+        if (ws_bytes < pl.ws_bytes) return TIDAR_ERR_WORKSPACE;
+    }
     AttnParams p;
     p.q = static_cast<const bf16 *>(q);
     p.k_new = static_cast<const bf16 *>(k_new);
@@ -98,7 +99,6 @@ tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new
     // grid is resident in one wave
     p.n_splits = attn_sm100_pick_splits(D, (long)B * Hkv * pl.mtiles, pl.max_tiles);
     p.Mpad = pl.Mpad;
-    p.part = static_cast<float *>(workspace);
     p.out = static_cast<bf16 *>(out);
     p.lse = lse;
     p.dev_status = dev_status;

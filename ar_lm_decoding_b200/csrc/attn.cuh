@@ -13,7 +13,6 @@ struct AttnParams {
     int mask_mode;
     int n_splits;      // key ranges per (sequence, KV head, row tile): the cluster size
     int Mpad;          // M rounded up to the row tile
-    float *part;       // [B*Hkv*Mpad/128][n_splits][128] partial-row records of 2D+16 bytes (workspace)
     bf16 *out;         // [B, R, Hq, D]
     float *lse;        // [B, R, Hq] or null
     int32_t *dev_status;

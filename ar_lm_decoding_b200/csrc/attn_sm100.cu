@@ -28,14 +28,15 @@
 // next S into those columns is issued after the PV that reads P, and
 // tcgen05.mma executes in issue order.
 // The CTAs that split one row tile's keys form a thread-block cluster.  At the
-// end the two warpgroups merge their states through shared memory (each
-// takes half of the columns) into one normalised partial row per query row,
-// stored as fp16 with a per-half-row fp32 scale (|error| <= 2^-12 of the row
-// maximum) and its log2 LSE in fp32; the CTA copies these records, coalesced,
-// to an L2-resident workspace.  After a cluster barrier (the only cross-CTA
-// wait, a hardware barrier) each CTA merges its slice of rows over the
-// cluster's S partials (LSE weights, fixed order) and writes the final bf16
-// output and LSE.
+// end each warpgroup combines its half of the columns of both O accumulators
+// straight from TMEM into one normalised partial row per query row, stored as
+// fp16 with a per-half-row fp32 scale (|error| <= 2^-12 of the row maximum)
+// and its log2 LSE in fp32.  With one split that row is the output.  Otherwise
+// the records are pushed over distributed shared memory into the idle K/V ring
+// of the cluster CTA that owns the row (a split cluster barrier: arrive once
+// the ring is idle, wait before pushing); after a second cluster barrier each
+// CTA merges its slice of rows over the S partials (LSE weights, fixed order)
+// and writes the final bf16 output and LSE.
 //
 // Every wait is bounded (clock64 budget); on expiry the CTA raises
 // TIDAR_DEV_TIMEOUT in dev_status, drains, frees TMEM and returns.
@@ -293,7 +294,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
         if (warp == 0 || warp == 2) {
             // ================= TMA producers: warp 0 streams K, warp 2 streams V =================
             // K of a tile is released as soon as its QK^T completes, V after its PV, so the K ring
@@ -365,14 +365,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
         __syncwarp();
-        tc::cluster_sync();  // every CTA of the cluster has written its partials
+        // the cluster barrier's two phases: rings idle (records may be pushed), records pushed
+        tc::cluster_arrive();
+        tc::cluster_wait();
+        tc::cluster_sync();
         if (warp == 1) {
             tc::fence_after_sync();
             tc::tmem_dealloc(tbase, 512);
         }
     } else {
         // ================= softmax warpgroups =================
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
         const int w = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
@@ -463,6 +465,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int v = 0; v < 2 && ok; ++v)  // both accumulators final (the ring is idle from here on)
             if (n > v) ok = tc::mbar_wait(o_done(v), 0, abort_flag, kWaitCycles);
         tc::fence_after_sync();
+        // this CTA's K/V ring is idle: once every CTA of the cluster has arrived here, the others may write
+        // their partial records into it (the wait is just before the push below)
+        tc::cluster_arrive();
         float *xml = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][2][TM]: m, l of each warpgroup
         xml[(w * 2 + 0) * TM + row] = n > w ? m_run : -INFINITY;
         xml[(w * 2 + 1) * TM + row] = n > w ? l_run : 0.f;
@@ -491,12 +496,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j) hv[c * 32 + j] = __uint_as_float(v0[j]) * f0 + __uint_as_float(v1[j]) * f1;
         }
         const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
-        const size_t group = (size_t)bh * (p.Mpad / TM) + mt;
-        // partial records of the row tile: vals [S][D/8][TM] (16 B = 8 fp16 per chunk: a warp's stores are
-        // contiguous), then hdr [S][TM] float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), 0)
-        uint8_t *gbase = reinterpret_cast<uint8_t *>(p.part) + group * S * TM * (2 * D + 16);
-        uint4 *vals = reinterpret_cast<uint4 *>(gbase);
-        float4 *hdr = reinterpret_cast<float4 *>(gbase + (size_t)S * TM * 2 * D);
+        // CTA s of the cluster merges rows [s*per, (s+1)*per) of the tile; it receives every CTA's partial
+        // record of those rows in its (idle) ring: vals [S][D/8][per] 16-byte chunks (8 fp16 of one row),
+        // then hdr [S][per] float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
+        const int per = ceil_div(TM, S);
+        uint8_t *recv = smem + L::KV_OFF + 4 * TM * sizeof(float);
+        uint4 *rvals = reinterpret_cast<uint4 *>(recv);
+        float4 *rhdr = reinterpret_cast<float4 *>(recv + (size_t)S * per * 2 * D);
+        uint4 pk[H / 8];
+        float scale = 1.f;
         if (S == 1) {  // the CTA saw every key of its rows: normalised output straight from the merge
             if (m_row < p.M) {
                 const size_t orow = (size_t)(b * p.R + r) * p.Hq + kvh * p.G + (m_row - r * p.G);
@@ -511,42 +519,44 @@ __global__ void __launch_bounds__(THREADS, 1)
             float amax = 0.f;
 #pragma unroll
             for (int j = 0; j < H; ++j) amax = fmaxf(amax, fabsf(hv[j]));
-            const float scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
+            scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
             const float rs = 1.f / scale;
-            uint4 *vrec = vals + ((size_t)split * (D / 8) + w * (H / 8)) * TM + row;
 #pragma unroll
             for (int j = 0; j < H / 8; ++j)
-                vrec[(size_t)j * TM] =
-                    make_uint4(pack_half2(hv[8 * j] * rs, hv[8 * j + 1] * rs), pack_half2(hv[8 * j + 2] * rs, hv[8 * j + 3] * rs),
-                               pack_half2(hv[8 * j + 4] * rs, hv[8 * j + 5] * rs), pack_half2(hv[8 * j + 6] * rs, hv[8 * j + 7] * rs));
-            float *h = reinterpret_cast<float *>(hdr + (size_t)split * TM + row);
-            h[1 + w] = scale;
-            if (w == 0) {
-                h[0] = lse2;
-                h[3] = 0.f;
-            }
+                pk[j] = make_uint4(pack_half2(hv[8 * j] * rs, hv[8 * j + 1] * rs), pack_half2(hv[8 * j + 2] * rs, hv[8 * j + 3] * rs),
+                                   pack_half2(hv[8 * j + 4] * rs, hv[8 * j + 5] * rs), pack_half2(hv[8 * j + 6] * rs, hv[8 * j + 7] * rs));
         }
-        // the records reach the other CTAs of the cluster through the barrier's release / acquire
+        tc::cluster_wait();  // every CTA's ring is idle
+        if (S > 1) {  // push this row's record to the CTA that merges it (consecutive lanes: consecutive chunks)
+            const int owner = row / per, rl = row - owner * per;
+            const uint32_t va = tc::cluster_map(smem_u32(rvals + ((size_t)split * (D / 8) + w * (H / 8)) * per + rl), owner);
+#pragma unroll
+            for (int j = 0; j < H / 8; ++j) tc::st_cluster_u32x4(va + j * per * 16, pk[j]);
+            const uint32_t ha = tc::cluster_map(smem_u32(rhdr + (size_t)split * per + rl), owner);
+            tc::st_cluster_f32(ha + 4 + 4 * w, scale);
+            if (w == 0) tc::st_cluster_f32(ha, lse2);
+        }
         tc::fence_before_sync();
-        tc::cluster_sync();
+        tc::cluster_sync();  // the records are in their owners' shared memory
 
         if (S > 1) {
-            // ---- merge this CTA's slice of rows over the cluster's S partial records (L2-resident) ----
-            // item = (16-byte column chunk c, row): consecutive threads take consecutive rows of one chunk, so
-            // every load below is coalesced; each thread issues all of an item's loads before using any
-            const int per = ceil_div(TM, S);
+            // ---- merge this CTA's rows over the cluster's S partial records (local shared memory) ----
             const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
             for (int it = tid - 128; it < nrows * (D / 8); it += 256) {
-                const int c = it / nrows, rr = row0 + (it - c * nrows);
+                const int c = it / nrows, rl = it - c * nrows;
                 float l2v[kMaxSplits], sc[kMaxSplits];
                 uint4 raw[kMaxSplits];
 #pragma unroll
-                for (int sp = 0; sp < kMaxSplits; ++sp) {  // unconditional loads (clamped index), masked below
-                    const int sq = min(sp, S - 1);
-                    const float4 hd = __ldcg(hdr + (size_t)sq * TM + rr);
-                    raw[sp] = __ldcg(vals + ((size_t)sq * (D / 8) + c) * TM + rr);
-                    l2v[sp] = sp < S ? hd.x : -INFINITY;
-                    sc[sp] = c < D / 16 ? hd.y : hd.z;
+                for (int sp = 0; sp < kMaxSplits; ++sp) {
+                    l2v[sp] = -INFINITY;
+                    sc[sp] = 0.f;
+                    raw[sp] = make_uint4(0, 0, 0, 0);
+                    if (sp < S) {
+                        const float4 hd = rhdr[sp * per + rl];
+                        raw[sp] = rvals[((size_t)sp * (D / 8) + c) * per + rl];
+                        l2v[sp] = hd.x;
+                        sc[sp] = c < D / 16 ? hd.y : hd.z;
+                    }
                 }
                 float mx = -INFINITY;
 #pragma unroll
@@ -567,7 +577,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         acc[2 * e + 1] += f * v.y;
                     }
                 }
-                const int m = mt * TM + rr;
+                const int m = mt * TM + row0 + rl;
                 if (m < p.M) {
                     const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
                     const int rq = m / p.G;

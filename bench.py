@@ -327,22 +327,25 @@ def gpu_arm(args, cfg):
     ms_step = ms / args.steps
     assert step.status.item() == 0
 
-    # dominant-kernel timing: each tidar_attn_step launch bracketed by events on its stream
-    n_attn = max(1, min(args.steps, 400)) * cfg.L
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(cfg.L)]
-    attn_ms = 0.0
-    reps = max(1, n_attn // cfg.L)
+    # dominant-kernel timing: the step's L tidar_attn_step launches captured alone in a graph on the same
+    # stream, replayed and timed with events on that stream (average launch duration as it runs in the step)
+    attn_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(attn_graph, stream=stream):
+        for l in range(cfg.L):
+            step.attn(l, stream.cuda_stream)
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 200))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         for _ in range(3):
-            step.run(stream.cuda_stream)
+            attn_graph.replay()
+        a0.record(stream)
         for _ in range(reps):
-            for l in range(cfg.L):
-                evs[l][0].record(stream)
-                step.attn(l, stream.cuda_stream)
-                evs[l][1].record(stream)
-            torch.cuda.synchronize()
-            attn_ms += sum(a.elapsed_time(b) for a, b in evs)
-    attn_ms_launch = max_over_ranks(attn_ms / (reps * cfg.L))
+            attn_graph.replay()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    attn_ms_launch = max_over_ranks(a0.elapsed_time(a1) / (reps * cfg.L))
+    del attn_graph
 
     # e2e: pinned host inputs copied in, the step, results read back, every step
     pin_in = torch.empty(step.in_bytes, dtype=torch.uint8, pin_memory=True)

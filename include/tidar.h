@@ -69,8 +69,10 @@ typedef enum {
 /* Attention                                                                 */
 /* ------------------------------------------------------------------------ */
 
-/* Bytes of workspace tidar_attn_step needs for these sizes (0 if invalid):
- * the split-KV partial rows, which stay L2-resident. */
+/* Bytes of device scratch tidar_attn_step needs for these sizes.  It is 0 for
+ * every size: the partial rows of the split-KV reduction pass between the CTAs
+ * of a thread-block cluster through distributed shared memory.  Invalid sizes
+ * are reported by tidar_attn_step itself. */
 size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max);
 
 /*
@@ -98,7 +100,7 @@ size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max
  * out        bf16 [B, R, Hq, D]  softmax(scale * q k^T) v over the visible keys
  * lse        f32  [B, R, Hq] or NULL: natural-log log-sum-exp of the scaled scores
  * workspace  >= tidar_attn_workspace_size(...) bytes of device memory, 256-byte
- *            aligned; its contents need no initialisation and are clobbered.
+ *            aligned; may be NULL (with ws_bytes 0) when that size is 0.
  * dev_status int32*; TIDAR_DEV_BAD_PREFIX set (and that sequence skipped) when
  *            a prefix length is out of range.
  * All tensor pointers must be 16-byte aligned.
