@@ -12,24 +12,26 @@
 //               from K_new/V_new through a 3-D tensor map (no head gather).
 //               A K stage is freed when its QK^T completes, a V stage when
 //               its PV does, so K runs ahead of V.
-//   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into the
-//               S columns of the warpgroup that owns the tile, then
-//               O += P V with P read from TMEM (tcgen05.mma A-from-TMEM).
-//   warps 4-7   softmax warpgroup 0: even tiles;  warps 8-11: odd tiles.
-//               Thread = query row = TMEM lane.  Each warpgroup keeps its
-//               own online-softmax state and its own O accumulator, so the
-//               tensor pipe computes one warpgroup's GEMMs while the other
-//               runs its exponentials.  The mask is evaluated from indices;
-//               O is rescaled only when the running max grows by more than
-//               2^8 (a stale max is exact as long as p <= 2^8 fits).
+//   warp 1      TMEM owner; one thread issues S = Q K^T (tcgen05.mma, both
+//               operands in shared memory) into S buffer j % 3.
+//   warp 3      one thread issues O += P V with P read from TMEM (A operand
+//               in TMEM, V an MN-major operand in shared memory).
+//   warps 4-11  softmax: both warpgroups work on every tile, warpgroup w on
+//               its columns [64w, 64w+64); thread = query row = TMEM lane.
+//               The two halves of a row agree on one running max through a
+//               small exchange in shared memory, so the exponentials of both
+//               halves share a scale and PV sums them into the one O.  The
+//               mask is evaluated from indices; O is rescaled only when the
+//               running max grows by more than 2^8 (a stale max is exact as
+//               long as p <= 2^8 fits).
 //   warps 2-3   also load Q when its rows cannot come through TMA.
-// TMEM (512 columns): warpgroup w owns S/P at [256w, 256w+128) and O at
-// [256w+128, 256w+128+D).  P (bf16) overwrites the first 64 columns of S; the
-// next S into those columns is issued after the PV that reads P, and
-// tcgen05.mma executes in issue order.
+// TMEM (512 columns): S buffers at [0, 128), [128, 256), [256, 384); O at
+// [384, 384+D).  P (bf16) overwrites the first 64 columns of its S buffer.
+// QK(j) reuses the buffer that PV(j-3) reads and is issued once PV(j-3) has
+// completed, so the softmax always has the next two tiles' S ready.
 // The CTAs that split one row tile's keys form a thread-block cluster.  At the
-// end each warpgroup combines its half of the columns of both O accumulators
-// straight from TMEM into one normalised partial row per query row, stored as
+// end each warpgroup reads its half of the columns of O from TMEM and forms
+// one normalised partial row per query row, stored as
 // fp16 with a per-half-row fp32 scale (|error| <= 2^-12 of the row maximum)
 // and its log2 LSE in fp32.  With one split that row is the output.  Otherwise
 // the records are pushed over distributed shared memory into the idle K/V ring
@@ -61,9 +63,11 @@ struct Smem {
     static constexpr int STAGE = 2 * KV_TILE;
     static constexpr int KV_OFF = Q_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
-    static constexpr int NBARS = 4 * STAGES + 7;  // k_full, k_empty, v_full, v_empty, s/p_full[2], o_done[2], q_full
+    // k_full, k_empty, v_full, v_empty, s_full[3], p_full[3], pv_done[2], o_final, q_full
+    static constexpr int NBARS = 4 * STAGES + 10;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-    static constexpr int TOTAL = MISC_OFF + 16;
+    static constexpr int XM_OFF = MISC_OFF + 16;      // row-max exchange between the warpgroups: [2][2][TM] bf16
+    static constexpr int TOTAL = XM_OFF + 2 * 2 * TM * 2;
     static constexpr int ALLOC = TOTAL + 1024;  // alignment slack
 };
 
@@ -96,23 +100,23 @@ __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv
     for (int kk = 0; kk < TN / 16; ++kk) tc::mma_ts(d_o, a_p + kk * 8, dv + kk * 128, id, (acc || kk > 0) ? 1u : 0u);
 }
 
-// Row maximum of the raw scores of one S tile (this thread's TMEM lane, TN columns).  MASKED: only keys
-// in [0, lo) and [glo, ghi) count.
+// Loads this thread's 64 raw scores (TMEM columns col .. col+63 of its lane) into x and returns their maximum.
+// MASKED: only keys kbase + j in [0, lo) and [glo, ghi) count (the others become -inf in x).
 template <bool MASKED>
-__device__ __forceinline__ float tile_max(uint32_t s_col, int lo, int glo, int ghi) {
-    float x[TN];
+__device__ __forceinline__ float half_load_max(uint32_t col, int kbase, int lo, int glo, int ghi, float (&x)[64]) {
 #pragma unroll
-    for (int c = 0; c < TN / 32; ++c) {
+    for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
-        tc::tmem_ld32(s_col + c * 32, v);
+        tc::tmem_ld32(col + c * 32, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) x[c * 32 + j] = __uint_as_float(v[j]);
     }
     tc::tmem_wait_ld();
     if constexpr (MASKED) {
 #pragma unroll
-        for (int c = 0; c < TN / 32; ++c) {
-            const uint32_t bits = range_bits(0, lo, c * 32) | range_bits(glo, ghi, c * 32);
+        for (int c = 0; c < 2; ++c) {
+            const int base = kbase + c * 32;
+            const uint32_t bits = range_bits(0, lo, base) | range_bits(glo, ghi, base);
 #pragma unroll
             for (int j = 0; j < 32; ++j) x[c * 32 + j] = (bits >> j) & 1u ? x[c * 32 + j] : -INFINITY;
         }
@@ -121,47 +125,129 @@ __device__ __forceinline__ float tile_max(uint32_t s_col, int lo, int glo, int g
 #pragma unroll
     for (int j = 0; j < 8; ++j) m8[j] = x[j];
 #pragma unroll
-    for (int j = 8; j < TN; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+    for (int j = 8; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
     return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
 
-// p = 2^(s * sl2 + neg_m) for one S tile, written back over S as bf16 pairs (P, the A operand of PV), in
-// 64-column chunks that re-read S from TMEM (a rolled loop keeps the code small).  Returns the row sum
-// of p.  Chunk c writes TMEM columns [32c, 32c + 32), which chunks > c do not read.
+// p = 2^(s * sl2 + neg_m) for the 64 scores in x, written as 32 bf16 pairs to TMEM columns pcol .. pcol+31
+// (P, the A operand of PV); masked-out keys give exactly 0.  Returns the sum of the 64 values of p.
 template <bool MASKED>
-__device__ __forceinline__ float tile_exp(uint32_t s_col, int lo, int glo, int ghi, float sl2, float neg_m) {
+__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], int kbase, int lo, int glo, int ghi,
+                                          float sl2, float neg_m) {
     float sum8[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < TN / 64; ++c) {
-        uint32_t v0[32], v1[32];
-        tc::tmem_ld32(s_col + c * 64, v0);
-        tc::tmem_ld32(s_col + c * 64 + 32, v1);
-        tc::tmem_wait_ld();
-        uint32_t bits0 = 0xffffffffu, bits1 = 0xffffffffu;
-        if constexpr (MASKED) {
-            bits0 = range_bits(0, lo, c * 64) | range_bits(glo, ghi, c * 64);
-            bits1 = range_bits(0, lo, c * 64 + 32) | range_bits(glo, ghi, c * 64 + 32);
-        }
-        uint32_t pk[32];
+    uint32_t bits[2] = {0xffffffffu, 0xffffffffu};
+    if constexpr (MASKED) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const uint32_t *v = j < 16 ? v0 : v1;
-            float a = fast_exp2(fmaf(__uint_as_float(v[(2 * j) & 31]), sl2, neg_m));
-            float bb = fast_exp2(fmaf(__uint_as_float(v[(2 * j + 1) & 31]), sl2, neg_m));
-            if constexpr (MASKED) {
-                const uint32_t bits = j < 16 ? bits0 : bits1;
-                a = (bits >> ((2 * j) & 31)) & 1u ? a : 0.f;
-                bb = (bits >> ((2 * j + 1) & 31)) & 1u ? bb : 0.f;
-            }
-            sum8[(2 * j) & 7] += a;
-            sum8[(2 * j + 1) & 7] += bb;
-            pk[j] = pack_bf16x2(a, bb);
-        }
-        tc::tmem_st32(s_col + c * 32, pk);
+        for (int c = 0; c < 2; ++c) bits[c] = range_bits(0, lo, kbase + c * 32) | range_bits(glo, ghi, kbase + c * 32);
     }
+    uint32_t pk[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        float a = fast_exp2(fmaf(x[2 * j], sl2, neg_m));
+        float bb = fast_exp2(fmaf(x[2 * j + 1], sl2, neg_m));
+        if constexpr (MASKED) {
+            a = (bits[j >> 4] >> ((2 * j) & 31)) & 1u ? a : 0.f;
+            bb = (bits[j >> 4] >> ((2 * j + 1) & 31)) & 1u ? bb : 0.f;
+        }
+        sum8[(2 * j) & 7] += a;
+        sum8[(2 * j + 1) & 7] += bb;
+        pk[j] = pack_bf16x2(a, bb);
+    }
+    tc::tmem_st32(pcol, pk);
     return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+}
+
+// Shared-memory layout of the split-KV exchange inside a CTA's (idle) K/V ring.  CTA s of an S-CTA cluster
+// merges rows [s*per, (s+1)*per) of the row tile, per = ceil(128 / S):
+//   [0, 4*TM floats)   the two warpgroups' (m, l) per row
+//   vals [S][D/8][per] 16-byte chunks (8 fp16 of one row, divided by the half-row scale)
+//   hdr  [S][per]      float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
+//   wts  [per][S][2]   merge weights of each split for the two column halves
+//   ost  [per][D + 8]  the merged rows, bf16 (row stride padded by 16 bytes)
+template <int D>
+struct Xchg {
+    uint8_t *base;
+    int S, per;
+    __device__ Xchg(uint8_t *ring, int S_, int per_) : base(ring + 4 * TM * sizeof(float)), S(S_), per(per_) {}
+    __device__ uint4 *vals() const { return reinterpret_cast<uint4 *>(base); }
+    __device__ float4 *hdr() const { return reinterpret_cast<float4 *>(base + (size_t)S * per * 2 * D); }
+    __device__ float *wts() const { return reinterpret_cast<float *>(base + (size_t)S * per * (2 * D + 16)); }
+    __device__ uint4 *ost() const {
+        return reinterpret_cast<uint4 *>(base + (size_t)S * per * (2 * D + 16) + align_up16((size_t)per * S * 8));
+    }
+    __device__ static size_t align_up16(size_t x) { return (x + 15) & ~size_t(15); }
+};
+
+// Merge of this CTA's rows over the S partial records of its cluster (all THREADS threads): the weights
+// exp2(lse_s - max) * scale / sum once per (row, split), then the weighted sum of the fp16 chunks, then the
+// merged rows copied out with each row's D*2 bytes written contiguously.
+template <int D, int S>
+__device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, int split, int mt, int b, int kvh,
+                                           int tid) {
+    constexpr int per = (TM + S - 1) / S, CH = D / 8;
+    const Xchg<D> x(ring, S, per);
+    const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
+    for (int rl = tid; rl < nrows; rl += THREADS) {
+        float4 hd[S];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) {
+            hd[sp] = x.hdr()[sp * per + rl];
+            mx = fmaxf(mx, hd[sp].x);
+        }
+        float wq[S], wsum = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) {
+            wq[sp] = hd[sp].x == -INFINITY ? 0.f : fast_exp2(hd[sp].x - mx);
+            wsum += wq[sp];
+        }
+        const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+        float2 *w = reinterpret_cast<float2 *>(x.wts()) + rl * S;
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) w[sp] = make_float2(wq[sp] * hd[sp].y * winv, wq[sp] * hd[sp].z * winv);
+        const int m = mt * TM + row0 + rl;
+        if (m < p.M && p.lse) {
+            const int rq = m / p.G;
+            p.lse[(size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G)] =
+                wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+        }
+    }
+    __syncthreads();
+    for (int it = tid; it < nrows * CH; it += THREADS) {  // consecutive threads: consecutive rows of chunk c
+        const int c = it / nrows, rl = it - c * nrows;
+        uint4 raw[S];
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) raw[sp] = x.vals()[(sp * CH + c) * per + rl];
+        const float2 *w = reinterpret_cast<const float2 *>(x.wts()) + rl * S;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) {
+            const float f = c < CH / 2 ? w[sp].x : w[sp].y;
+            const uint32_t u[4] = {raw[sp].x, raw[sp].y, raw[sp].z, raw[sp].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 v = unpack_half2(u[e]);
+                acc[2 * e] = fmaf(f, v.x, acc[2 * e]);
+                acc[2 * e + 1] = fmaf(f, v.y, acc[2 * e + 1]);
+            }
+        }
+        x.ost()[rl * (CH + 1) + c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+    __syncthreads();
+    for (int it = tid; it < nrows * CH; it += THREADS) {  // consecutive threads: consecutive chunks of a row
+        const int rl = it / CH, c = it - rl * CH;
+        const int m = mt * TM + row0 + rl;
+        if (m < p.M) {
+            const int rq = m / p.G;
+            const size_t orow = (size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G);
+            *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) = x.ost()[rl * (CH + 1) + c];
+        }
+    }
 }
 
 // Number of valid keys in tile t (t < TP: prefix tile, else new-key tile).
@@ -185,10 +271,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto k_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto v_full = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
     auto v_empty = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
-    auto s_full = [&](int w) { return bar0 + 8u * (4 * STAGES + w); };
-    auto p_full = [&](int w) { return bar0 + 8u * (4 * STAGES + 2 + w); };
-    auto o_done = [&](int w) { return bar0 + 8u * (4 * STAGES + 4 + w); };
-    const uint32_t q_full = bar0 + 8u * (4 * STAGES + 6);
+    auto s_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + sb); };      // S buffer sb holds a new S
+    auto p_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + 3 + sb); };  // P in S buffer sb is complete
+    // pv_done(e): its k-th phase completes with PV(2k + e).  Waiting for PV(i) on pv_done(i & 1) is unambiguous
+    // once PV(i-2) has completed, which holds wherever it is waited for (see there).
+    auto pv_done = [&](int e) { return bar0 + 8u * (4 * STAGES + 6 + e); };
+    const uint32_t o_final = bar0 + 8u * (4 * STAGES + 8);  // one phase: the last PV has completed
+    const uint32_t q_full = bar0 + 8u * (4 * STAGES + 9);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -203,11 +292,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mbar_init(v_full(s), 1);
             tc::mbar_init(v_empty(s), 1);
         }
-        for (int w = 0; w < 2; ++w) {
-            tc::mbar_init(s_full(w), 1);
-            tc::mbar_init(p_full(w), 128);
-            tc::mbar_init(o_done(w), 1);
+        for (int sb = 0; sb < 3; ++sb) {
+            tc::mbar_init(s_full(sb), 1);
+            tc::mbar_init(p_full(sb), 256);  // both softmax warpgroups
         }
+        tc::mbar_init(pv_done(0), 1);
+        tc::mbar_init(pv_done(1), 1);
+        tc::mbar_init(o_final, 1);
         tc::mbar_init(q_full, q_tma ? 1 : THREADS - 64);
         *abort_flag = 0;
         tc::mbar_fence_init();
@@ -217,11 +308,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::tma_prefetch_desc(&tm_vn);
     }
     if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
-    // every global read below (prefix lengths, Q, K/V, the workspace) waits for the previous kernel
+    // every global read below (prefix lengths, Q, K/V) waits for the previous kernel
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    if (tid == 0) {
+        // Q does not depend on the prefix length: its copy starts at once
+        if (q_tma) {  // rows (r, g) of the tile: box {64 d, G heads, 128/G rows}
+            tc::mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+                tc::tma_load_3d(sQ + h * TM * 128, &tm_q, h * 64, kvh * p.G, b * p.R + mt * (TM / p.G), q_full);
+        }
+    }
     const int P = p.prefix_len[b];
     if (P < 0 || P > p.P_max) {
         if (tid == 0 && split == 0 && mt == 0) atomicOr(p.dev_status, TIDAR_DEV_BAD_PREFIX);
+        if (tid == 0 && q_tma) tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);  // no copy may land after exit
         tc::fence_before_sync();
         __syncthreads();
         if (warp == 1) {
@@ -258,12 +359,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---- thread 0 starts the first copies at once ----
     const int prologue = min(n, STAGES);
     if (tid == 0) {
-        if (q_tma) {  // rows (r, g) of the tile: box {64 d, G heads, 128/G rows}
-            tc::mbar_arrive_expect_tx(q_full, L::Q_BYTES);
-#pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-                tc::tma_load_3d(sQ + h * TM * 128, &tm_q, h * 64, kvh * p.G, b * p.R + mt * (TM / p.G), q_full);
-        }
         for (int i = 0; i < prologue; ++i) {
             issue_tile(i, 0);
             issue_tile(i, 1);
@@ -315,51 +410,59 @@ __global__ void __launch_bounds__(THREADS, 1)
                                   kWaitCycles);
             }
             __syncwarp();
-        } else if (warp == 1) {
-            // ================= MMA issuer: one thread runs the whole loop =================
-            // Order: QK(0), QK(1), then PV(i), QK(i+2) for every i -- QK(i+2) writes the S/P columns that
-            // PV(i) reads, and tcgen05.mma executes in issue order.  The loop has no warp-wide operation and
-            // no division: its thread spends its time in barrier waits and MMA issue.
-            if (lane == 0) {
+        } else if (warp == 1 || warp == 3) {
+            // ================= MMA issue: QK^T on warp 1, PV on warp 3 (one thread each) =================
+            // Two issuing threads on two SM sub-partitions: each issues half of a tile's MMAs, so neither's
+            // issue rate bounds the tensor pipe.  S of tile j goes to S buffer j % 3.  QK(j), j >= 3, reuses the
+            // buffer whose P PV(j-3) reads, so it is issued once PV(j-3) has completed; with three S buffers that
+            // costs nothing, since the softmax still has S(j-2) and S(j-1) to work on.
+            constexpr uint64_t kStage = L::STAGE >> 4;  // one ring stage in the descriptor's address field
+            const uint32_t tb = tbase;
+            if (lane == 0 && warp == 1) {
                 constexpr uint32_t id_qk = tc::idesc_bf16_f32(TM, TN, 0, 0);
-                constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
-                constexpr uint64_t kStage = L::STAGE >> 4;  // one ring stage in the descriptor's address field
                 // descriptors are built once; a k-step or stage moves the start address, which lives in the
                 // low 14 bits (address >> 4; shared memory is < 256 KB, so the add never carries out)
                 const uint64_t dq = tc::smem_desc_sw128(sQ, 16, 1024);
                 const uint64_t dk = tc::smem_desc_sw128(sKV, 16, 1024);
-                const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
-                const uint32_t tb = tbase;
                 bool ok = tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);
-                int kst = 0, vst = 0;       // ring stages of the next QK and the next PV
-                uint32_t kph = 0, vph = 0;  // and the phase parities they wait for
-                for (int it = 0; ok && it < n + 2; ++it) {
-                    if (it >= 2) {  // PV(i), i = it - 2
-                        const int i = it - 2, w = i & 1;
-                        ok = tc::mbar_wait(v_full(vst), vph, abort_flag, kWaitCycles) &&
-                             tc::mbar_wait(p_full(w), (i >> 1) & 1, abort_flag, kWaitCycles);
+                int kst = 0;
+                uint32_t kph = 0;
+                for (int j = 0; j < n && ok; ++j) {
+                    const int sb = j % 3;
+                    if (j >= 3) {  // PV(j-3) done reading P from buffer sb (PV(j-5) was waited for before)
+                        ok = tc::mbar_wait(pv_done((j - 3) & 1), ((j - 3) >> 1) & 1, abort_flag, kWaitCycles);
                         if (!ok) break;
-                        tc::fence_after_sync();
-                        issue_pv<D>(tb + w * 256 + 128, tb + w * 256, dv + vst * kStage, id_pv, i >= 2);
-                        tc::mma_commit(v_empty(vst));
-                        if (i + 2 >= n) tc::mma_commit(o_done(w));
-                        if (++vst == STAGES) {
-                            vst = 0;
-                            vph ^= 1u;
-                        }
                     }
-                    if (it < n) {  // QK(it)
-                        const int w = it & 1;
-                        ok = tc::mbar_wait(k_full(kst), kph, abort_flag, kWaitCycles);
-                        if (!ok) break;
-                        tc::fence_after_sync();
-                        issue_qk<D>(tb + w * 256, dq, dk + kst * kStage, id_qk);
-                        tc::mma_commit(s_full(w));
-                        tc::mma_commit(k_empty(kst));
-                        if (++kst == STAGES) {
-                            kst = 0;
-                            kph ^= 1u;
-                        }
+                    ok = tc::mbar_wait(k_full(kst), kph, abort_flag, kWaitCycles);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    issue_qk<D>(tb + sb * 128, dq, dk + kst * kStage, id_qk);
+                    tc::mma_commit(s_full(sb));
+                    tc::mma_commit(k_empty(kst));
+                    if (++kst == STAGES) {
+                        kst = 0;
+                        kph ^= 1u;
+                    }
+                }
+            } else if (lane == 0 && warp == 3) {
+                constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
+                const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
+                bool ok = true;
+                int vst = 0;
+                uint32_t vph = 0;
+                for (int i = 0; i < n && ok; ++i) {
+                    const int sb = i % 3;
+                    ok = tc::mbar_wait(v_full(vst), vph, abort_flag, kWaitCycles) &&
+                         tc::mbar_wait(p_full(sb), (i / 3) & 1, abort_flag, kWaitCycles);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    issue_pv<D>(tb + 384, tb + sb * 128, dv + vst * kStage, id_pv, i > 0);
+                    tc::mma_commit(v_empty(vst));
+                    tc::mma_commit(pv_done(i & 1));
+                    if (i == n - 1) tc::mma_commit(o_final);
+                    if (++vst == STAGES) {
+                        vst = 0;
+                        vph ^= 1u;
                     }
                 }
             }
@@ -374,12 +477,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::tmem_dealloc(tbase, 512);
         }
     } else {
-        // ================= softmax warpgroups =================
+        // ================= softmax: both warpgroups on every tile =================
+        // Warpgroup w takes columns [64w, 64w+64) of each S tile (thread = query row = TMEM lane).  The two
+        // halves of a row agree on one running max through a small exchange in shared memory, so both scale
+        // their exponentials alike and PV sums them into the one O accumulator.
         const int w = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int m_row = mt * TM + row;
         const int r = m_row / p.G;
+        const int wt = tid - 128;  // 0..255
         // visible new keys of row r: [0, vis_lim) and [vis_glo, vis_ghi) (same rule as new_key_visible)
         int vis_lim, vis_glo = 0, vis_ghi = 0;
         if (p.mask_mode == TIDAR_MASK_CAUSAL || r < p.k) {
@@ -391,14 +498,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             vis_ghi = vis_glo + p.k;
         }
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const uint32_t s_col = tbase + lane_off + w * 256;
-        const uint32_t o_col = s_col + 128;
+        const uint32_t o_col = tbase + lane_off + 384 + w * (D / 2);  // this warpgroup's half of O
+        __nv_bfloat16 *xm = reinterpret_cast<__nv_bfloat16 *>(smem + L::XM_OFF);  // [2 tiles][2 wg][TM]
         const float sl2 = p.scale_log2;  // > 0, so the max of raw scores gives the max of scaled ones
-        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units) and sum
+        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units, shared by both halves), own sum
         bool ok = true;
-        for (int i = w; i < n; i += 2) {
-            if (!tc::mbar_wait(s_full(w), (i >> 1) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
+        for (int i = 0; i < n; ++i) {
+            const int sb = i % 3;
+            if (!tc::mbar_wait(s_full(sb), (i / 3) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
             tc::fence_after_sync();
+            const uint32_t s_col = tbase + lane_off + sb * 128;
             const int t = t0 + i;
             // a partial prefix tile (keys beyond P) or a new-key tile (the TiDAR mask): the visible keys of
             // this row are [0, lo) and [glo, ghi); everything else, garbage included, is excluded by select
@@ -418,13 +527,29 @@ __global__ void __launch_bounds__(THREADS, 1)
                 lo = min(lo, end);
                 ghi = min(ghi, end);
             }
-            const float mx = (masked ? tile_max<true>(s_col, lo, glo, ghi) : tile_max<false>(s_col, lo, glo, ghi)) * sl2;
+            float x[64];
+            const float hmx = masked ? half_load_max<true>(s_col + w * 64, w * 64, lo, glo, ghi, x)
+                                     : half_load_max<false>(s_col + w * 64, w * 64, lo, glo, ghi, x);
+            // both halves' maxima (rounded to bf16 for the exchange: any value the two sides agree on and that
+            // is within 2^8 of the true maximum serves, since p = 2^(s - m) then fits comfortably)
+            const __nv_bfloat16 hb = __float2bfloat16_rn(hmx);
+            xm[((i & 1) * 2 + w) * TM + row] = hb;
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");
+            const __nv_bfloat16 ob = xm[((i & 1) * 2 + (1 - w)) * TM + row];
+            const float mx = fmaxf(__bfloat162float(hb), __bfloat162float(ob)) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + 8.f;
-            if (i >= 2 && __any_sync(0xffffffffu, grow)) {  // rescale O (last written by the PV of tile i-2)
+            if (i >= 1 && __any_sync(0xffffffffu, grow)) {
+                // rescale this half of O once PV(i-1), the last to write it, has completed.  S(i) is complete, and
+                // QK(i) was issued after PV(i-3), so PV(i-3) has completed: the wait below is unambiguous.
+                if (!tc::mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, kWaitCycles)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
                 const float f = grow ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t v[32];
                     tc::tmem_ld32(o_col + c * 32, v);
                     tc::tmem_wait_ld();
@@ -438,14 +563,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 m_run = m_new;
             }
             const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-            l_run += masked ? tile_exp<true>(s_col, lo, glo, ghi, sl2, neg_m) : tile_exp<false>(s_col, lo, glo, ghi, sl2, neg_m);
+            // P of keys [64w, 64w+64) into S columns [32w, 32w+32): both halves' S loads precede the exchange
+            l_run += masked ? half_exp<true>(s_col + w * 32, x, w * 64, lo, glo, ghi, sl2, neg_m)
+                            : half_exp<false>(s_col + w * 32, x, w * 64, lo, glo, ghi, sl2, neg_m);
             const int valid = tile_valid(t, TP, P, p.R);
             if (valid < TN) {
                 // keys past the sequence: zero their V rows (0 * garbage could be NaN) before PV reads them
                 const int st = i % STAGES;
                 if (!tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
                 uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
-                for (int idx = row; idx < (TN - valid) * (D / 8); idx += 128) {
+                for (int idx = wt; idx < (TN - valid) * (D / 8); idx += 256) {
                     const int j = valid + idx / (D / 8), c = idx % (D / 8);
                     *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
                         make_uint4(0, 0, 0, 0);
@@ -454,47 +581,38 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            tc::mbar_arrive(p_full(w));
+            tc::mbar_arrive(p_full(sb));
         }
         // the next kernel in the stream may launch now: it waits for this grid before touching memory
         asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-        // ---- merge the two warpgroups' states.  A thread may read every TMEM column of its lane quadrant, so
-        // warpgroup w combines columns [w*D/2, (w+1)*D/2) of BOTH O accumulators straight from TMEM; only the
-        // row statistics (m, l) pass through shared memory ----
         constexpr int H = D / 2;
-        for (int v = 0; v < 2 && ok; ++v)  // both accumulators final (the ring is idle from here on)
-            if (n > v) ok = tc::mbar_wait(o_done(v), 0, abort_flag, kWaitCycles);
+        if (ok && n > 0) ok = tc::mbar_wait(o_final, 0, abort_flag, kWaitCycles);  // O final
         tc::fence_after_sync();
         // this CTA's K/V ring is idle: once every CTA of the cluster has arrived here, the others may write
         // their partial records into it (the wait is just before the push below)
         tc::cluster_arrive();
-        float *xml = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][2][TM]: m, l of each warpgroup
-        xml[(w * 2 + 0) * TM + row] = n > w ? m_run : -INFINITY;
-        xml[(w * 2 + 1) * TM + row] = n > w ? l_run : 0.f;
+        // the row sum is split over the two halves
+        float *xl = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM]
+        xl[w * TM + row] = l_run;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        const float m0 = xml[row], l0 = xml[TM + row], m1 = xml[2 * TM + row], l1 = xml[3 * TM + row];
-        const float mm = fmaxf(m0, m1);
-        const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
-        const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
-        const float lt = l0 * a0 + l1 * a1;
+        const float lt = l_run + xl[(1 - w) * TM + row];
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float lse2 = lt > 0.f ? mm + __log2f(lt) : -INFINITY;  // log2 of this CTA's row sum
-        // tcgen05.ld is warp-collective: the decision to read an accumulator must be warp-uniform
-        const bool rd0 = __all_sync(0xffffffffu, ok && n > 0), rd1 = __all_sync(0xffffffffu, ok && n > 1);
-        const float f0 = rd0 ? a0 * inv : 0.f, f1 = rd1 ? a1 * inv : 0.f;
-        const uint32_t o0 = tbase + lane_off + 128 + w * H, o1 = tbase + lane_off + 256 + 128 + w * H;
-        float hv[H];
+        const float lse2 = lt > 0.f ? m_run + __log2f(lt) : -INFINITY;  // log2 of this CTA's row sum
+        // tcgen05.ld is warp-collective: the decision to read the accumulator must be warp-uniform
+        const bool rd = __all_sync(0xffffffffu, ok && n > 0);
+        uint32_t va[H / 32][32];
 #pragma unroll
         for (int c = 0; c < H / 32; ++c) {
-            uint32_t v0[32], v1[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0u;
-            if (rd0) tc::tmem_ld32(o0 + c * 32, v0);
-            if (rd1) tc::tmem_ld32(o1 + c * 32, v1);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) hv[c * 32 + j] = __uint_as_float(v0[j]) * f0 + __uint_as_float(v1[j]) * f1;
+            for (int j = 0; j < 32; ++j) va[c][j] = 0u;
+            if (rd) tc::tmem_ld32(o_col + c * 32, va[c]);
         }
+        tc::tmem_wait_ld();
+        float hv[H];
+#pragma unroll
+        for (int c = 0; c < H / 32; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) hv[c * 32 + j] = rd ? __uint_as_float(va[c][j]) * inv : 0.f;
         const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
         // CTA s of the cluster merges rows [s*per, (s+1)*per) of the tile; it receives every CTA's partial
         // record of those rows in its (idle) ring: vals [S][D/8][per] 16-byte chunks (8 fp16 of one row),
@@ -516,9 +634,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (w == 0 && p.lse) p.lse[orow] = lse2 * kLn2;
             }
         } else {
-            float amax = 0.f;
+            float am[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-            for (int j = 0; j < H; ++j) amax = fmaxf(amax, fabsf(hv[j]));
+            for (int j = 0; j < H; ++j) am[j & 3] = fmaxf(am[j & 3], fabsf(hv[j]));
+            const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
             scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
             const float rs = 1.f / scale;
 #pragma unroll
@@ -529,66 +648,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::cluster_wait();  // every CTA's ring is idle
         if (S > 1) {  // push this row's record to the CTA that merges it (consecutive lanes: consecutive chunks)
             const int owner = row / per, rl = row - owner * per;
-            const uint32_t va = tc::cluster_map(smem_u32(rvals + ((size_t)split * (D / 8) + w * (H / 8)) * per + rl), owner);
+            const uint32_t ra = tc::cluster_map(smem_u32(rvals + ((size_t)split * (D / 8) + w * (H / 8)) * per + rl), owner);
 #pragma unroll
-            for (int j = 0; j < H / 8; ++j) tc::st_cluster_u32x4(va + j * per * 16, pk[j]);
+            for (int j = 0; j < H / 8; ++j) tc::st_cluster_u32x4(ra + j * per * 16, pk[j]);
             const uint32_t ha = tc::cluster_map(smem_u32(rhdr + (size_t)split * per + rl), owner);
             tc::st_cluster_f32(ha + 4 + 4 * w, scale);
             if (w == 0) tc::st_cluster_f32(ha, lse2);
         }
         tc::fence_before_sync();
         tc::cluster_sync();  // the records are in their owners' shared memory
+    }
 
-        if (S > 1) {
-            // ---- merge this CTA's rows over the cluster's S partial records (local shared memory) ----
-            const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
-            for (int it = tid - 128; it < nrows * (D / 8); it += 256) {
-                const int c = it / nrows, rl = it - c * nrows;
-                float l2v[kMaxSplits], sc[kMaxSplits];
-                uint4 raw[kMaxSplits];
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplits; ++sp) {
-                    l2v[sp] = -INFINITY;
-                    sc[sp] = 0.f;
-                    raw[sp] = make_uint4(0, 0, 0, 0);
-                    if (sp < S) {
-                        const float4 hd = rhdr[sp * per + rl];
-                        raw[sp] = rvals[((size_t)sp * (D / 8) + c) * per + rl];
-                        l2v[sp] = hd.x;
-                        sc[sp] = c < D / 16 ? hd.y : hd.z;
-                    }
-                }
-                float mx = -INFINITY;
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplits; ++sp) mx = fmaxf(mx, l2v[sp]);
-                float acc[8], wsum = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplits; ++sp) {
-                    const float wq = l2v[sp] == -INFINITY ? 0.f : fast_exp2(l2v[sp] - mx);
-                    wsum += wq;
-                    const float f = wq * sc[sp];
-                    const uint32_t u[4] = {raw[sp].x, raw[sp].y, raw[sp].z, raw[sp].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 v = unpack_half2(u[e]);
-                        acc[2 * e] += f * v.x;
-                        acc[2 * e + 1] += f * v.y;
-                    }
-                }
-                const int m = mt * TM + row0 + rl;
-                if (m < p.M) {
-                    const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
-                    const int rq = m / p.G;
-                    const size_t orow = (size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G);
-                    *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) =
-                        make_uint4(pack_bf16x2(acc[0] * winv, acc[1] * winv), pack_bf16x2(acc[2] * winv, acc[3] * winv),
-                                   pack_bf16x2(acc[4] * winv, acc[5] * winv), pack_bf16x2(acc[6] * winv, acc[7] * winv));
-                    if (c == 0 && p.lse) p.lse[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
-                }
-            }
-        }
+    // ---- merge this CTA's rows over the cluster's S partial records (local shared memory, all threads) ----
+    switch (p.n_splits) {
+        case 2: merge_rows<D, 2>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        case 3: merge_rows<D, 3>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        case 4: merge_rows<D, 4>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        case 5: merge_rows<D, 5>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        case 6: merge_rows<D, 6>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        case 7: merge_rows<D, 7>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        case 8: merge_rows<D, 8>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
+        default: break;  // one split: the output was written by the warpgroup merge
     }
     if (tid == 0 && *abort_flag) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
 }
