@@ -164,7 +164,6 @@ __device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], i
 //   [0, 4*TM floats)   the two warpgroups' (m, l) per row
 //   vals [S][D/8][per] 16-byte chunks (8 fp16 of one row, divided by the half-row scale)
 //   hdr  [S][per]      float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
-//   wts  [per][S][2]   merge weights of each split for the two column halves
 //   ost  [per][D + 8]  the merged rows, bf16 (row stride padded by 16 bytes)
 template <int D>
 struct Xchg {
@@ -173,60 +172,39 @@ struct Xchg {
     __device__ Xchg(uint8_t *ring, int S_, int per_) : base(ring + 4 * TM * sizeof(float)), S(S_), per(per_) {}
     __device__ uint4 *vals() const { return reinterpret_cast<uint4 *>(base); }
     __device__ float4 *hdr() const { return reinterpret_cast<float4 *>(base + (size_t)S * per * 2 * D); }
-    __device__ float *wts() const { return reinterpret_cast<float *>(base + (size_t)S * per * (2 * D + 16)); }
-    __device__ uint4 *ost() const {
-        return reinterpret_cast<uint4 *>(base + (size_t)S * per * (2 * D + 16) + align_up16((size_t)per * S * 8));
-    }
-    __device__ static size_t align_up16(size_t x) { return (x + 15) & ~size_t(15); }
+    __device__ uint4 *ost() const { return reinterpret_cast<uint4 *>(base + (size_t)S * per * (2 * D + 16)); }
 };
 
-// Merge of this CTA's rows over the S partial records of its cluster (all THREADS threads): the weights
-// exp2(lse_s - max) * scale / sum once per (row, split), then the weighted sum of the fp16 chunks, then the
-// merged rows copied out with each row's D*2 bytes written contiguously.
+// Merge of this CTA's rows over the S partial records of its cluster (all THREADS threads): item = (16-byte
+// column chunk, row), consecutive threads on consecutive rows of one chunk; each item weighs the S chunks by
+// exp2(lse_s - max) * scale_s / sum, then the merged rows are copied out with each row's D*2 bytes written
+// contiguously.
 template <int D, int S>
 __device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, int split, int mt, int b, int kvh,
                                            int tid) {
     constexpr int per = (TM + S - 1) / S, CH = D / 8;
     const Xchg<D> x(ring, S, per);
     const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
-    for (int rl = tid; rl < nrows; rl += THREADS) {
+    for (int it = tid; it < nrows * CH; it += THREADS) {
+        const int c = it / nrows, rl = it - c * nrows;
         float4 hd[S];
-        float mx = -INFINITY;
+        uint4 raw[S];
 #pragma unroll
         for (int sp = 0; sp < S; ++sp) {
             hd[sp] = x.hdr()[sp * per + rl];
-            mx = fmaxf(mx, hd[sp].x);
+            raw[sp] = x.vals()[(sp * CH + c) * per + rl];
         }
-        float wq[S], wsum = 0.f;
+        float mx = -INFINITY;
 #pragma unroll
-        for (int sp = 0; sp < S; ++sp) {
-            wq[sp] = hd[sp].x == -INFINITY ? 0.f : fast_exp2(hd[sp].x - mx);
-            wsum += wq[sp];
-        }
-        const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
-        float2 *w = reinterpret_cast<float2 *>(x.wts()) + rl * S;
-#pragma unroll
-        for (int sp = 0; sp < S; ++sp) w[sp] = make_float2(wq[sp] * hd[sp].y * winv, wq[sp] * hd[sp].z * winv);
-        const int m = mt * TM + row0 + rl;
-        if (m < p.M && p.lse) {
-            const int rq = m / p.G;
-            p.lse[(size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G)] =
-                wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
-        }
-    }
-    __syncthreads();
-    for (int it = tid; it < nrows * CH; it += THREADS) {  // consecutive threads: consecutive rows of chunk c
-        const int c = it / nrows, rl = it - c * nrows;
-        uint4 raw[S];
-#pragma unroll
-        for (int sp = 0; sp < S; ++sp) raw[sp] = x.vals()[(sp * CH + c) * per + rl];
-        const float2 *w = reinterpret_cast<const float2 *>(x.wts()) + rl * S;
-        float acc[8];
+        for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, hd[sp].x);
+        float acc[8], wsum = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int sp = 0; sp < S; ++sp) {
-            const float f = c < CH / 2 ? w[sp].x : w[sp].y;
+            const float wq = hd[sp].x == -INFINITY ? 0.f : fast_exp2(hd[sp].x - mx);
+            wsum += wq;
+            const float f = wq * (c < CH / 2 ? hd[sp].y : hd[sp].z);
             const uint32_t u[4] = {raw[sp].x, raw[sp].y, raw[sp].z, raw[sp].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -235,8 +213,16 @@ __device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, i
                 acc[2 * e + 1] = fmaf(f, v.y, acc[2 * e + 1]);
             }
         }
-        x.ost()[rl * (CH + 1) + c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                                pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+        x.ost()[rl * (CH + 1) + c] =
+            make_uint4(pack_bf16x2(acc[0] * winv, acc[1] * winv), pack_bf16x2(acc[2] * winv, acc[3] * winv),
+                       pack_bf16x2(acc[4] * winv, acc[5] * winv), pack_bf16x2(acc[6] * winv, acc[7] * winv));
+        const int m = mt * TM + row0 + rl;
+        if (c == 0 && m < p.M && p.lse) {
+            const int rq = m / p.G;
+            p.lse[(size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G)] =
+                wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+        }
     }
     __syncthreads();
     for (int it = tid; it < nrows * CH; it += THREADS) {  // consecutive threads: consecutive chunks of a row
@@ -468,10 +454,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
         __syncwarp();
-        // the cluster barrier's two phases: rings idle (records may be pushed), records pushed
-        tc::cluster_arrive();
+        // the cluster barrier's two phases: rings idle (records may be pushed), records pushed.  These warps
+        // publish nothing, so their arrivals carry no release fence.
+        tc::cluster_arrive_relaxed();
         tc::cluster_wait();
-        tc::cluster_sync();
+        tc::cluster_arrive_relaxed();
+        tc::cluster_wait();
         if (warp == 1) {
             tc::fence_after_sync();
             tc::tmem_dealloc(tbase, 512);
@@ -589,8 +577,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ok && n > 0) ok = tc::mbar_wait(o_final, 0, abort_flag, kWaitCycles);  // O final
         tc::fence_after_sync();
         // this CTA's K/V ring is idle: once every CTA of the cluster has arrived here, the others may write
-        // their partial records into it (the wait is just before the push below)
-        tc::cluster_arrive();
+        // their partial records into it (the wait is just before the push below).  The arrival publishes
+        // nothing, so it carries no release fence.
+        tc::cluster_arrive_relaxed();
         // the row sum is split over the two halves
         float *xl = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM]
         xl[w * TM + row] = l_run;
