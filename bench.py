@@ -531,6 +531,50 @@ def reference_arm(args, cfg):
     }
 
 
+def attn_prefix_sweep(args, cfg):
+    """Attention time per launch against the prefix length at a fixed P_max (so a fixed split count): the
+    intercept of the line is the per-launch fixed cost (set-up, first copies, epilogue), the slope the cost
+    of one more key tile of a row tile.  One JSON line per prefix length, then the fit."""
+    import torch
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    step = Step(cfg, device)
+    stream = torch.cuda.Stream(device)
+    pts = []
+    for P in sorted({min(cfg.P_max, x) for x in (128, 1024, 2048, 3072, 4096)}):
+        step.prefix.fill_(P)
+        with torch.cuda.stream(stream):
+            for l in range(cfg.L):
+                step.attn(l, stream.cuda_stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for l in range(cfg.L):
+                step.attn(l, stream.cuda_stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                g.replay()
+            e0.record(stream)
+            reps = max(3, min(args.steps, 50))
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * cfg.L)
+        tiles = math.ceil(P / 128) + math.ceil(cfg.R / 128)
+        pts.append((tiles, us))
+        print(json.dumps({"mode": "attn_prefix_sweep", "workload": cfg.name, "prefix": P, "key_tiles": tiles,
+                          "us_per_launch": round(us, 3), "status": int(step.status.item())}), flush=True)
+        del g
+    n = len(pts)
+    mx = sum(t for t, _ in pts) / n
+    my = sum(u for _, u in pts) / n
+    slope = sum((t - mx) * (u - my) for t, u in pts) / max(1e-9, sum((t - mx) ** 2 for t, _ in pts))
+    print(json.dumps({"mode": "attn_prefix_sweep_fit", "workload": cfg.name, "fixed_us": round(my - slope * mx, 3),
+                      "us_per_key_tile": round(slope, 4)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -540,6 +584,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--attn-prefix-sweep", action="store_true",
+                    help="print attention time per launch against the prefix length (not the benchmark line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -551,6 +597,9 @@ def main():
         import oracle
         oracle.build()
         print(json.dumps(reference_arm(args, cfg)), flush=True)
+        return
+    if args.attn_prefix_sweep:
+        attn_prefix_sweep(args, cfg)
         return
     res = gpu_arm(args, cfg)
     if res is not None:
