@@ -100,10 +100,10 @@ __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv
     for (int kk = 0; kk < TN / 16; ++kk) tc::mma_ts(d_o, a_p + kk * 8, dv + kk * 128, id, (acc || kk > 0) ? 1u : 0u);
 }
 
-// Loads this thread's 64 raw scores (TMEM columns col .. col+63 of its lane) into x and returns their maximum.
-// MASKED: only keys kbase + j in [0, lo) and [glo, ghi) count (the others become -inf in x).
+// Loads this thread's 64 raw scores (TMEM columns col .. col+63 of its lane) into x.  MASKED: only keys
+// kbase + j in [0, lo) and [glo, ghi) are kept; the others (garbage past the sequence included) become -inf.
 template <bool MASKED>
-__device__ __forceinline__ float half_load_max(uint32_t col, int kbase, int lo, int glo, int ghi, float (&x)[64]) {
+__device__ __forceinline__ void half_load(uint32_t col, int kbase, int lo, int glo, int ghi, float (&x)[64]) {
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
@@ -121,6 +121,9 @@ __device__ __forceinline__ float half_load_max(uint32_t col, int kbase, int lo, 
             for (int j = 0; j < 32; ++j) x[c * 32 + j] = (bits >> j) & 1u ? x[c * 32 + j] : -INFINITY;
         }
     }
+}
+
+__device__ __forceinline__ float half_max(const float (&x)[64]) {
     float m8[8];  // eight independent chains
 #pragma unroll
     for (int j = 0; j < 8; ++j) m8[j] = x[j];
@@ -129,33 +132,29 @@ __device__ __forceinline__ float half_load_max(uint32_t col, int kbase, int lo, 
     return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
 
-// p = 2^(s * sl2 + neg_m) for the 64 scores in x, written as 32 bf16 pairs to TMEM columns pcol .. pcol+31
-// (P, the A operand of PV); masked-out keys give exactly 0.  Returns the sum of the 64 values of p.
-template <bool MASKED>
-__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], int kbase, int lo, int glo, int ghi,
-                                          float sl2, float neg_m) {
-    float sum8[8];
+// p = 2^(x * sl2 + neg_m) for the 64 scores in x (-inf gives exactly 0), written as 32 bf16 pairs to TMEM
+// columns pcol .. pcol+31 (P, the A operand of PV).  Returns the sum of the 64 values of p; *mx receives the
+// maximum of x, computed in the same pass (its ALU work hides under the exponentials).
+__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], float sl2, float neg_m, float *mx) {
+    float sum8[8], m8[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
-    uint32_t bits[2] = {0xffffffffu, 0xffffffffu};
-    if constexpr (MASKED) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) bits[c] = range_bits(0, lo, kbase + c * 32) | range_bits(glo, ghi, kbase + c * 32);
+    for (int j = 0; j < 8; ++j) {
+        sum8[j] = 0.f;
+        m8[j] = -INFINITY;
     }
     uint32_t pk[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-        float a = fast_exp2(fmaf(x[2 * j], sl2, neg_m));
-        float bb = fast_exp2(fmaf(x[2 * j + 1], sl2, neg_m));
-        if constexpr (MASKED) {
-            a = (bits[j >> 4] >> ((2 * j) & 31)) & 1u ? a : 0.f;
-            bb = (bits[j >> 4] >> ((2 * j + 1) & 31)) & 1u ? bb : 0.f;
-        }
+        const float a = fast_exp2(fmaf(x[2 * j], sl2, neg_m));
+        const float bb = fast_exp2(fmaf(x[2 * j + 1], sl2, neg_m));
+        m8[(2 * j) & 7] = fmaxf(m8[(2 * j) & 7], x[2 * j]);
+        m8[(2 * j + 1) & 7] = fmaxf(m8[(2 * j + 1) & 7], x[2 * j + 1]);
         sum8[(2 * j) & 7] += a;
         sum8[(2 * j + 1) & 7] += bb;
         pk[j] = pack_bf16x2(a, bb);
     }
     tc::tmem_st32(pcol, pk);
+    *mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
     return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 }
 
@@ -516,10 +515,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ghi = min(ghi, end);
             }
             float x[64];
-            const float hmx = masked ? half_load_max<true>(s_col + w * 64, w * 64, lo, glo, ghi, x)
-                                     : half_load_max<false>(s_col + w * 64, w * 64, lo, glo, ghi, x);
+            if (masked)
+                half_load<true>(s_col + w * 64, w * 64, lo, glo, ghi, x);
+            else
+                half_load<false>(s_col + w * 64, w * 64, lo, glo, ghi, x);
+            // Exponentials against the running max the two halves already share (stale by design: exact as long
+            // as p <= 2^8); the tile's row max comes out of the same pass.  Only a row whose max grew by more
+            // than 2^8 -- all rows on the first tile, rarely later -- redoes them with the new max.
+            const uint32_t pcol = s_col + w * 32;  // P of keys [64w, 64w+64) over S columns [32w, 32w+32)
+            const bool fresh = m_run == -INFINITY;  // no visible key so far: no max to reuse
+            float hmx;
+            float lt = fresh ? 0.f : half_exp(pcol, x, sl2, -m_run, &hmx);
+            if (fresh) hmx = half_max(x);
             // both halves' maxima (rounded to bf16 for the exchange: any value the two sides agree on and that
-            // is within 2^8 of the true maximum serves, since p = 2^(s - m) then fits comfortably)
+            // is within 2^8 of the true maximum serves)
             const __nv_bfloat16 hb = __float2bfloat16_rn(hmx);
             xm[((i & 1) * 2 + w) * TM + row] = hb;
             asm volatile("bar.sync 1, 256;\n" ::: "memory");
@@ -527,33 +536,35 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float mx = fmaxf(__bfloat162float(hb), __bfloat162float(ob)) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool grow = m_new > m_run + 8.f;
-            if (i >= 1 && __any_sync(0xffffffffu, grow)) {
-                // rescale this half of O once PV(i-1), the last to write it, has completed.  S(i) is complete, and
-                // QK(i) was issued after PV(i-3), so PV(i-3) has completed: the wait below is unambiguous.
-                if (!tc::mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, kWaitCycles)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const float f = grow ? fast_exp2(m_run - m_new) : 1.f;
+            if (__any_sync(0xffffffffu, grow || fresh)) {  // fresh rows have written no P yet
+                if (i >= 1 && __any_sync(0xffffffffu, grow)) {
+                    // rescale this half of O once PV(i-1), the last to write it, has completed.  S(i) is
+                    // complete, and QK(i) was issued after PV(i-3) completed: the wait below is unambiguous.
+                    if (!tc::mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, kWaitCycles)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const float f = grow ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll 1
-                for (int c = 0; c < D / 64; ++c) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(o_col + c * 32, v);
-                    tc::tmem_wait_ld();
+                    for (int c = 0; c < D / 64; ++c) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(o_col + c * 32, v);
+                        tc::tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-                    tc::tmem_st32(o_col + c * 32, v);
+                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+                        tc::tmem_st32(o_col + c * 32, v);
+                    }
                 }
+                if (grow) {
+                    l_run *= fast_exp2(m_run - m_new);
+                    m_run = m_new;
+                }
+                tc::tmem_wait_st();  // the redone P overwrites the first pass's
+                float unused;
+                lt = half_exp(pcol, x, sl2, m_run == -INFINITY ? 0.f : -m_run, &unused);
             }
-            if (grow) {
-                l_run *= fast_exp2(m_run - m_new);
-                m_run = m_new;
-            }
-            const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-            // P of keys [64w, 64w+64) into S columns [32w, 32w+32): both halves' S loads precede the exchange
-            l_run += masked ? half_exp<true>(s_col + w * 32, x, w * 64, lo, glo, ghi, sl2, neg_m)
-                            : half_exp<false>(s_col + w * 32, x, w * 64, lo, glo, ghi, sl2, neg_m);
+            l_run += lt;
             const int valid = tile_valid(t, TP, P, p.R);
             if (valid < TN) {
                 // keys past the sequence: zero their V rows (0 * garbage could be NaN) before PV reads them
