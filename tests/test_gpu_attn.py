@@ -89,6 +89,40 @@ def test_full_size_sampled_rows(name):
     assert eo <= O_TOL and el <= LSE_TOL, (name, eo, el)
 
 
+def _plant_growing_spikes(cfg, inp, step_nat):
+    """For every 128-key tile t of the cache and every KV head, overwrite one key so that it scores
+    (4 + step_nat * t) natural-log units against one query row of that head's group (a different row each
+    tile, the key in column 37 t mod 128 so both column halves get spikes).  The running max of those rows
+    grows by ~step_nat / ln 2 log2-units on every tile -- more than the 2^8 stale-max allowance -- while the
+    other rows of the same warps do not grow."""
+    q = synth.bf16_bits_to_f32(inp["q"]).astype(np.float64)
+    kc = synth.bf16_bits_to_f32(inp["k_cache"]).copy()
+    G = cfg.Hq // cfg.Hkv
+    scale = 1.0 / np.sqrt(cfg.D)
+    for b in range(cfg.B):
+        P = int(inp["prefix_len"][b])
+        for h in range(cfg.Hkv):
+            for t in range((P + 127) // 128):
+                n = t * 128 + (37 * t) % 128
+                if n >= P:
+                    continue
+                r, g = t % cfg.R, h * G + (t % G)
+                qv = q[b, r, g]
+                target = 4.0 + step_nat * t
+                kc[b, h, n] = (qv * (target / (scale * float(qv @ qv)))).astype(np.float32)
+    out = dict(inp)
+    out["k_cache"] = synth.f32_to_bf16_bits(kc)
+    return out
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,P", [(1, 8, 2, 2000), (2, 4, 1, 1200)])
+def test_running_max_growth_rescales(B, Hq, Hkv, P):
+    # every tile raises some rows' maxima by ~10 log2-units: the rescale of O and the redone exponentials
+    cfg = TINY.with_(B=B, Hq=Hq, Hkv=Hkv, D=128, k=3, P=P)
+    inp = _plant_growing_spikes(cfg, synth.make_attn_inputs(cfg, seed=7), step_nat=7.0)
+    _check_full(cfg, inp=inp)
+
+
 def test_group_rows_ignore_later_drafts_bitwise():
     cfg = TINY.with_(k=4, P=190, Hq=4, Hkv=2)
     k = cfg.k
