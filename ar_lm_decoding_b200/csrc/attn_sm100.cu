@@ -160,24 +160,24 @@ __device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], f
 
 // Shared-memory layout of the split-KV exchange inside a CTA's (idle) K/V ring.  CTA s of an S-CTA cluster
 // merges rows [s*per, (s+1)*per) of the row tile, per = ceil(128 / S):
-//   [0, 4*TM floats)   the two warpgroups' (m, l) per row
-//   vals [S][D/8][per] 16-byte chunks (8 fp16 of one row, divided by the half-row scale)
-//   hdr  [S][per]      float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
-//   ost  [per][D + 8]  the merged rows, bf16 (row stride padded by 16 bytes)
+//   [0, 4*TM floats)    row statistics exchanged between the warpgroups
+//   vals [S][D/8][pv]   16-byte chunks (8 fp16 of one row, divided by the half-row scale); pv = per rounded up
+//                       to an odd number, so that reading one chunk of consecutive rows and reading the
+//                       consecutive chunks of one row both spread over all shared-memory banks
+//   hdr  [S][per]       float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
 template <int D>
 struct Xchg {
     uint8_t *base;
-    int S, per;
-    __device__ Xchg(uint8_t *ring, int S_, int per_) : base(ring + 4 * TM * sizeof(float)), S(S_), per(per_) {}
+    int S, per, pv;
+    __device__ Xchg(uint8_t *ring, int S_, int per_)
+        : base(ring + 4 * TM * sizeof(float)), S(S_), per(per_), pv(per_ | 1) {}
     __device__ uint4 *vals() const { return reinterpret_cast<uint4 *>(base); }
-    __device__ float4 *hdr() const { return reinterpret_cast<float4 *>(base + (size_t)S * per * 2 * D); }
-    __device__ uint4 *ost() const { return reinterpret_cast<uint4 *>(base + (size_t)S * per * (2 * D + 16)); }
+    __device__ float4 *hdr() const { return reinterpret_cast<float4 *>(base + (size_t)S * pv * 2 * D); }
 };
 
-// Merge of this CTA's rows over the S partial records of its cluster (all THREADS threads): item = (16-byte
-// column chunk, row), consecutive threads on consecutive rows of one chunk; each item weighs the S chunks by
-// exp2(lse_s - max) * scale_s / sum, then the merged rows are copied out with each row's D*2 bytes written
-// contiguously.
+// Merge of this CTA's rows over the S partial records of its cluster (all THREADS threads): item = (row,
+// 16-byte column chunk), consecutive threads on consecutive chunks of one row, so that every warp writes whole
+// output rows; each item weighs the S chunks by exp2(lse_s - max) * scale_s / sum.
 template <int D, int S>
 __device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, int split, int mt, int b, int kvh,
                                            int tid) {
@@ -185,13 +185,13 @@ __device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, i
     const Xchg<D> x(ring, S, per);
     const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
     for (int it = tid; it < nrows * CH; it += THREADS) {
-        const int c = it / nrows, rl = it - c * nrows;
+        const int rl = it / CH, c = it - rl * CH;
         float4 hd[S];
         uint4 raw[S];
 #pragma unroll
         for (int sp = 0; sp < S; ++sp) {
             hd[sp] = x.hdr()[sp * per + rl];
-            raw[sp] = x.vals()[(sp * CH + c) * per + rl];
+            raw[sp] = x.vals()[(sp * CH + c) * x.pv + rl];
         }
         float mx = -INFINITY;
 #pragma unroll
@@ -212,25 +212,15 @@ __device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, i
                 acc[2 * e + 1] = fmaf(f, v.y, acc[2 * e + 1]);
             }
         }
-        const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
-        x.ost()[rl * (CH + 1) + c] =
-            make_uint4(pack_bf16x2(acc[0] * winv, acc[1] * winv), pack_bf16x2(acc[2] * winv, acc[3] * winv),
-                       pack_bf16x2(acc[4] * winv, acc[5] * winv), pack_bf16x2(acc[6] * winv, acc[7] * winv));
-        const int m = mt * TM + row0 + rl;
-        if (c == 0 && m < p.M && p.lse) {
-            const int rq = m / p.G;
-            p.lse[(size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G)] =
-                wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
-        }
-    }
-    __syncthreads();
-    for (int it = tid; it < nrows * CH; it += THREADS) {  // consecutive threads: consecutive chunks of a row
-        const int rl = it / CH, c = it - rl * CH;
         const int m = mt * TM + row0 + rl;
         if (m < p.M) {
+            const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
             const int rq = m / p.G;
             const size_t orow = (size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G);
-            *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) = x.ost()[rl * (CH + 1) + c];
+            *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) =
+                make_uint4(pack_bf16x2(acc[0] * winv, acc[1] * winv), pack_bf16x2(acc[2] * winv, acc[3] * winv),
+                           pack_bf16x2(acc[4] * winv, acc[5] * winv), pack_bf16x2(acc[6] * winv, acc[7] * winv));
+            if (c == 0 && p.lse) p.lse[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
         }
     }
 }
@@ -618,9 +608,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // record of those rows in its (idle) ring: vals [S][D/8][per] 16-byte chunks (8 fp16 of one row),
         // then hdr [S][per] float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
         const int per = ceil_div(TM, S);
-        uint8_t *recv = smem + L::KV_OFF + 4 * TM * sizeof(float);
-        uint4 *rvals = reinterpret_cast<uint4 *>(recv);
-        float4 *rhdr = reinterpret_cast<float4 *>(recv + (size_t)S * per * 2 * D);
+        const Xchg<D> xc(smem + L::KV_OFF, S, per);
         uint4 pk[H / 8];
         float scale = 1.f;
         if (S == 1) {  // the CTA saw every key of its rows: normalised output straight from the merge
@@ -648,10 +636,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::cluster_wait();  // every CTA's ring is idle
         if (S > 1) {  // push this row's record to the CTA that merges it (consecutive lanes: consecutive chunks)
             const int owner = row / per, rl = row - owner * per;
-            const uint32_t ra = tc::cluster_map(smem_u32(rvals + ((size_t)split * (D / 8) + w * (H / 8)) * per + rl), owner);
+            const uint32_t ra =
+                tc::cluster_map(smem_u32(xc.vals() + ((size_t)split * (D / 8) + w * (H / 8)) * xc.pv + rl), owner);
 #pragma unroll
-            for (int j = 0; j < H / 8; ++j) tc::st_cluster_u32x4(ra + j * per * 16, pk[j]);
-            const uint32_t ha = tc::cluster_map(smem_u32(rhdr + (size_t)split * per + rl), owner);
+            for (int j = 0; j < H / 8; ++j) tc::st_cluster_u32x4(ra + j * xc.pv * 16, pk[j]);
+            const uint32_t ha = tc::cluster_map(smem_u32(xc.hdr() + (size_t)split * per + rl), owner);
             tc::st_cluster_f32(ha + 4 + 4 * w, scale);
             if (w == 0) tc::st_cluster_f32(ha, lse2);
         }
