@@ -49,7 +49,9 @@ def workload_desc(cfg, B):
 
 
 def algorithmic_bytes(cfg, prefix_sum):
-    """Compulsory HBM bytes of one step (measurement section)."""
+    """Compulsory HBM bytes of one step: every cached K/V row of every layer read once, the step's own
+    Q/K_new/V_new read and O/LSE written once per layer, and the vocabulary rows the verify and the draft
+    selection must read (p, q and the k slot rows of group j*)."""
     B, L, R = cfg.B, cfg.L, cfg.R
     es = 2 if cfg.logits_dtype == "bf16" else 4
     kv = 4 * L * cfg.Hkv * cfg.D * prefix_sum                    # K and V cache rows, bf16
