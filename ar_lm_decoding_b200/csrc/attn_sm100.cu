@@ -18,12 +18,14 @@
 //               in TMEM, V an MN-major operand in shared memory).
 //   warps 4-11  softmax: both warpgroups work on every tile, warpgroup w on
 //               its columns [64w, 64w+64); thread = query row = TMEM lane.
-//               The two halves of a row agree on one running max through a
-//               small exchange in shared memory, so the exponentials of both
-//               halves share a scale and PV sums them into the one O.  The
-//               mask is evaluated from indices; O is rescaled only when the
-//               running max grows by more than 2^8 (a stale max is exact as
-//               long as p <= 2^8 fits).
+//               The two halves of a row always hold the same running max,
+//               so their exponentials share a scale and PV sums them into
+//               the one O.  A tile is exponentiated against that (possibly
+//               stale) max -- exact as long as p <= 2^8 fits -- while its row
+//               max is taken in the same pass; the halves then exchange
+//               maxima through shared memory, and only rows whose max grew
+//               by more than 2^8 redo their exponentials and rescale O.  The
+//               mask is evaluated from indices.
 //   warps 2-3   also load Q when its rows cannot come through TMA.
 // TMEM (512 columns): S buffers at [0, 128), [128, 256), [256, 384); O at
 // [384, 384+D).  P (bf16) overwrites the first 64 columns of its S buffer.
