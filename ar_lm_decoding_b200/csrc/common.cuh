@@ -17,7 +17,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kNumSMs = 148;
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
-__host__ __device__ __forceinline__ int round_up(int a, int b) { return ceil_div(a, b) * b; }
 __host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Visibility of new key nn (0..R-1, same order as the query rows) to query
@@ -35,12 +34,6 @@ __device__ __forceinline__ bool new_key_visible(int mask_mode, int k, int r, int
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 

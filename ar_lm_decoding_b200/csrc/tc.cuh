@@ -151,12 +151,8 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
-// The two halves of cluster_sync(), for work that fits between them.
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-}
-// Arrival that publishes nothing (no release fence): for threads whose earlier writes the other CTAs do
-// not read after the barrier.
+// The two halves of cluster_sync(), for work that fits between them.  The arrival publishes nothing (no
+// release fence): for threads whose earlier writes the other CTAs do not read after the barrier.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
 }

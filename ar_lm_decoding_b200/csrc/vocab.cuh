@@ -9,7 +9,6 @@ namespace tidar {
 
 constexpr int kChunk = 8192;        // vocabulary entries per CTA
 constexpr int kStatThreads = 256;   // kChunk / kStatThreads = 32 entries per thread
-constexpr int kScanThreads = 1024;  // kChunk / kScanThreads = 8 entries per thread
 
 struct ChunkStat {
     float m;   // max logit of the chunk
@@ -64,10 +63,6 @@ __device__ __forceinline__ void load_chunk32(const void *row, int dtype, int V, 
     }
 }
 
-__device__ __forceinline__ int chunk_entry_index(int c, int e) {
-    return c * kChunk + (e >> 3) * 2048 + threadIdx.x * 8 + (e & 7);
-}
-
 // Block-wide max (blockDim.x == kStatThreads).  `red` holds >= 8 floats.
 __device__ __forceinline__ float block_max256(float v, float *red) {
     v = warp_max(v);
@@ -112,59 +107,6 @@ __device__ __forceinline__ ChunkStat chunk_stat(const void *row, int dtype, int 
     st.pad = 0.f;
     st.z = block_sum_d<kStatThreads>((double)s, redd);
     return st;
-}
-
-// Merge chunk statistics in chunk order: returns max m and sum exp(x - m).
-__device__ __forceinline__ void merge_stats(const ChunkStat *st, int n, float &m, double &z) {
-    m = -INFINITY;
-    for (int c = 0; c < n; ++c) m = fmaxf(m, st[c].m);
-    z = 0.0;
-    for (int c = 0; c < n; ++c)
-        if (st[c].m != -INFINITY) z += st[c].z * exp2((double)(st[c].m - m) * 1.4426950408889634);
-}
-
-// Inclusive prefix scan over the kScanThreads x 8 weights of one chunk, then
-// the first local index whose inclusive sum exceeds `target` (or, when
-// rounding leaves none, the last index with positive weight).  `w` holds this
-// thread's 8 consecutive weights (entries tid*8 .. tid*8+7 of the chunk).
-__device__ __forceinline__ int chunk_search(const double (&w)[8], double target, double *scan_buf, int *pick) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    double loc = 0.0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) loc += w[e];
-    // warp inclusive scan of the per-thread totals
-    double incl = loc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const double y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (tid == 0) { pick[0] = 0x7fffffff; pick[1] = -1; }
-    if (lane == 31) scan_buf[warp] = incl;
-    __syncthreads();
-    if (tid == 0) {
-        double run = 0.0;
-        for (int i = 0; i < kScanThreads / 32; ++i) {
-            const double t = scan_buf[i];
-            scan_buf[i] = run;
-            run += t;
-        }
-    }
-    __syncthreads();
-    double c = scan_buf[warp] + incl - loc;  // exclusive prefix of this thread
-    int first = 0x7fffffff, last = -1;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        c += w[e];
-        if (w[e] > 0.0) {
-            last = tid * 8 + e;
-            if (c > target && first == 0x7fffffff) first = tid * 8 + e;
-        }
-    }
-    if (first != 0x7fffffff) atomicMin(&pick[0], first);
-    if (last >= 0) atomicMax(&pick[1], last);
-    __syncthreads();
-    return pick[0] != 0x7fffffff ? pick[0] : pick[1];
 }
 
 // This thread's 32 consecutive entries (tid*32 .. tid*32+31) of chunk c (256 threads), -inf beyond V.
@@ -248,13 +190,6 @@ __device__ __forceinline__ void merge_stats_warp(const ChunkStat *st, int n, flo
     for (int c = lane; c < n; c += 32)
         if (st[c].m != -INFINITY) s += st[c].z * (double)exp2f((st[c].m - m) * kLog2e);
     z = warp_sum_d(s);
-}
-
-// This thread's 8 consecutive entries (tid*8..tid*8+7) of chunk c as floats (-inf beyond V).
-__device__ __forceinline__ void load_chunk8(const void *row, int dtype, int V, int c, float (&v)[8]) {
-    const int i0 = c * kChunk + threadIdx.x * 8;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = i0 + e < V ? load_logit(row, dtype, (size_t)(i0 + e)) : -INFINITY;
 }
 
 }  // namespace tidar
