@@ -98,27 +98,34 @@ class ClockSampler:
             self.proc.kill()
         self.file.flush()
         with open(self.file.name) as f:
-            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+            text = f.read()
         os.unlink(self.file.name)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            r = [x.strip() for x in r]
-            if len(r) < 9:
-                continue
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, r[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm_sorted = sorted(sm)
-        return {"sm_mhz": sm_sorted[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return parse_clock_samples(text)
+
+
+def parse_clock_samples(text):
+    """Median SM clock, max SM clock and the throttle reasons seen in nvidia-smi CSV samples of
+    ClockSampler.QUERY (no header, no units)."""
+    rows = [r.split(",") for r in text.strip().splitlines() if r.strip()]
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        r = [x.strip() for x in r]
+        if len(r) < 9:
+            continue
+        try:
+            sm.append(float(r[1]))
+            mx.append(float(r[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, r[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+    sm_sorted = sorted(sm)
+    return {"sm_mhz": sm_sorted[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm)}
 
 
 # ---------------------------------------------------------------------------
