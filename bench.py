@@ -268,6 +268,34 @@ def gpu_smi_id(device):
         return str(device.index or 0)
 
 
+class Ranks:
+    """The replicas of a multi-GPU run (one process per GPU, torch.distributed initialised by the caller):
+    a barrier and the maximum of a per-rank time, so that every figure is the slowest rank's."""
+
+    def __init__(self, world, device=None):
+        self.world, self.device = world, device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x):
+        if self.world == 1:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def job_throughput(world, step_s):
+    """Whole-job steps/s: each of the `world` replicas completes one step every `step_s` seconds (the slowest
+    rank's step time)."""
+    return world / step_s
+
+
 def kernels_per_step(cfg):
     # per layer: one attention kernel (split-KV merged in-kernel); verify: 2 (vocab statistics, decision);
     # commit: 1 (its counters are zeroed by a memset node, not a kernel)
@@ -288,16 +316,8 @@ def gpu_arm(args, cfg):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, device)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     step = Step(cfg, device, seed=rank)
     stream = torch.cuda.Stream(device)
@@ -387,7 +407,7 @@ def gpu_arm(args, cfg):
     attn_bytes_launch = (byts["kv"] + byts["qkvo"]) / cfg.L
     achieved = attn_bytes_launch / (attn_ms_launch / 1e3) / 1e9
     traffic = load_traffic(cfg)
-    value = world / step_s  # every rank completes one step per step_s
+    value = job_throughput(world, step_s)
     res = {
         "metric": METRIC,
         "value": round(value, 3),
