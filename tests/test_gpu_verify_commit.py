@@ -112,7 +112,8 @@ def _commit_inputs(cfg, seed, L=3):
     return kc, vc, kn, vn, pl, al, rs, v["group_logits"], v["u_draft"]
 
 
-@pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k4", "qwen3-8b_k8_b8", "qwen2.5-1.5b_k16"])
+@pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k4", "qwen2.5-1.5b_k16", "qwen3-8b_k8", "qwen3-8b_k8_b8",
+                                  "qwen3-32b_k16"])
 def test_commit_parity(name):
     cfg = synth.CONFIGS[name]
     report = []
