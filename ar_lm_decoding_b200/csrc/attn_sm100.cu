@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const Xchg<D> xc(smem + L::KV_OFF, S, per);
         uint4 pk[H / 8];
         float scale = 1.f;
-        if (S == 1) {  // the CTA saw every key of its rows: normalised output straight from the merge
+        if (S == 1) {  // the CTA saw every key of its rows: the normalised half row is the output
             if (m_row < p.M) {
                 const size_t orow = (size_t)(b * p.R + r) * p.Hq + kvh * p.G + (m_row - r * p.G);
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + w * H);
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         case 6: merge_rows<D, 6>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
         case 7: merge_rows<D, 7>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
         case 8: merge_rows<D, 8>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        default: break;  // one split: the output was written by the warpgroup merge
+        default: break;  // one split: each warpgroup wrote its half of every output row directly
     }
     if (tid == 0 && *abort_flag) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
 }
