@@ -73,6 +73,22 @@ struct Smem {
     static constexpr int ALLOC = TOTAL + 1024;  // alignment slack
 };
 
+static_assert(Smem<64>::ALLOC <= 227 * 1024 && Smem<128>::ALLOC <= 227 * 1024, "shared memory beyond 227 KB");
+
+// Bytes the split-KV exchange of an S-CTA cluster uses at the start of a CTA's (idle) K/V ring: the row
+// statistics, the S partial records of its rows (row stride rounded up to an odd number of chunks) and their
+// headers.
+constexpr int xchg_bytes(int S, int D) {
+    const int per = (TM + S - 1) / S;
+    return 4 * TM * 4 + S * (per | 1) * 2 * D + S * per * 16;
+}
+constexpr bool xchg_fits(int D) {
+    for (int S = 2; S <= kMaxSplits; ++S)
+        if (xchg_bytes(S, D) > STAGES * 2 * TN * D * 2) return false;  // the K and V rings
+    return true;
+}
+static_assert(xchg_fits(64) && xchg_fits(128), "split-KV exchange larger than the K/V ring");
+
 // Bit i set iff key base+i lies in [a, b) (i = 0..31).
 __device__ __forceinline__ uint32_t range_bits(int a, int b, int base) {
     const int lo = max(a - base, 0), hi = min(b - base, 32);
