@@ -16,8 +16,6 @@ cudaError_t commit_launch(void *const *, void *const *, const void *const *, con
 
 namespace {
 
-constexpr int kMaxDraft = 16;
-
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
 

@@ -183,15 +183,56 @@ def test_commit_accept_zero_writes_nothing():
 
 
 def test_draft_sampling_hand_worked_inverse_cdf():
+    # the token and its interval of the normalised CDF: the interval decides which GPU/oracle differences are
+    # exempt, so it is pinned to the hand-worked values as well
     z = np.log(np.array([0.25, 0.25, 0.5], np.float64)).astype(np.float32)
     rows = read_golden("inverse_cdf_hand.txt")
     k = 1
-    for u, tok in rows:
+    for u, tok, lo, hi in rows:
         g = np.broadcast_to(z, (1, k + 1, k, 3)).copy()
         _, kc, vc, kn, vn, pl = _commit_case(L=1, B=1, Hkv=1, D=2, k=k, P=4)
         out = oracle.kv_commit(kc, vc, kn, vn, pl, np.array([1], np.int32), np.array([-1], np.int32), g,
                                np.array([[float(u)]], np.float32))
         assert out["next_drafts"][0, 0] == int(tok), (u, tok)
+        assert abs(out["draft_lo"][0, 0] - float(lo)) < 1e-6 and abs(out["draft_hi"][0, 0] - float(hi)) < 1e-6
+
+
+def test_draft_interval_is_undefined_for_the_resampled_slot():
+    # after a rejection slot 0 is the resampled token, not a draw: no interval, so no exemption can apply
+    z = np.log(np.array([0.25, 0.25, 0.5], np.float64)).astype(np.float32)
+    k = 2
+    g = np.broadcast_to(z, (1, k + 1, k, 3)).copy()
+    _, kc, vc, kn, vn, pl = _commit_case(L=1, B=1, Hkv=1, D=2, k=k, P=4)
+    out = oracle.kv_commit(kc, vc, kn, vn, pl, np.array([1], np.int32), np.array([2], np.int32), g,
+                           np.array([[0.3, 0.3]], np.float32))
+    assert out["next_drafts"][0, 0] == 2 and np.isnan(out["draft_lo"][0, 0]) and np.isnan(out["draft_hi"][0, 0])
+    assert out["next_drafts"][0, 1] == 1 and abs(out["draft_lo"][0, 1] - 0.25) < 1e-6
+
+
+def test_residual_resample_hand_worked_interval():
+    p = np.log(np.array([0.4, 0.1, 0.3, 0.2]))
+    q = np.log(np.array([0.1, 0.3, 0.2, 0.4]))
+    for u, tok, lo, hi in read_golden("residual_cdf_hand.txt"):
+        inp = _verify_inputs(p[None, None], q[None, None], [[1]], [[0.5]], [float(u)])
+        out = oracle.verify(inp)
+        assert out["accept_len"][0] == 0 and abs(out["ratio"][0, 0] - 1 / 3) < 1e-6
+        assert out["resampled"][0] == int(tok), (u, tok)
+        assert abs(out["res_lo"][0] - float(lo)) < 1e-6 and abs(out["res_hi"][0] - float(hi)) < 1e-6
+    # every draft accepted: no resample, no interval
+    inp = _verify_inputs(p[None, None], q[None, None], [[0]], [[0.5]], [0.5])
+    out = oracle.verify(inp)
+    assert out["accept_len"][0] == 1 and out["resampled"][0] == -1
+    assert np.isnan(out["res_lo"][0]) and np.isnan(out["res_hi"][0])
+
+
+def test_residual_interval_when_p_equals_q_falls_back_to_p():
+    # p == q leaves no residual mass (unreachable in exact arithmetic after a rejection, but forced here):
+    # the draw falls back to p itself, and the interval is p's CDF interval
+    p = np.log(np.array([0.5, 0.25, 0.25]))
+    inp = _verify_inputs(p[None, None], p[None, None], [[2]], [[0.5]], [0.6])
+    out = oracle.verify(inp, forced_accept_len=np.array([0], np.int32))
+    assert out["resampled"][0] == 1
+    assert abs(out["res_lo"][0] - 0.5) < 1e-6 and abs(out["res_hi"][0] - 0.75) < 1e-6
 
 
 def test_draft_sampling_follows_group_softmax():
