@@ -5,14 +5,20 @@
 Prints one JSON line (rank 0).  The default workload is the Qwen3-8B-shaped
 step (36 layers, 32 query / 8 KV heads, head dim 128, cached prefix 4096,
 draft length 8 -> 80 query rows per layer, vocabulary 151936, batch 1).
-Inputs are synthetic (seeded, generated on the device); every layer has its
-own KV cache, so a step reads ~0.6 GB, far more than the 126 MB L2.
+Inputs are synthetic and seeded: Q/K/V and the KV caches are drawn on the
+device, the logits, drafts and uniforms by the numpy recipe the parity tests
+use.  Every layer has its own KV cache, so a step reads ~0.6 GB, far more
+than the 126 MB L2.
 
 Timing: the step is captured in a CUDA graph (layers stay separate launches);
 W warm-up replays, then K timed replays between CUDA events on the launching
 stream, with a barrier and device synchronise on both sides; the max over
-ranks is reported.  With N > 1 every rank runs an independent replica (the
-path has no cross-GPU exchange), so scaling is weak.
+ranks is reported.  `e2e` runs the same step through the C ABI without a
+graph, every step copying its inputs from pinned host memory and reading its
+results back on the host (host wall clock).  With --gpus N > 1 the script
+starts N replicas itself (torchrun, one process per GPU) unless a launcher
+already did; every rank runs an independent replica (the path has no
+cross-GPU exchange), so scaling is weak.
 """
 from __future__ import annotations
 
@@ -136,6 +142,7 @@ class Step:
     """Device-resident inputs and outputs of one decode step, and its launches."""
 
     def __init__(self, cfg, device, seed=0):
+        import numpy as np
         import torch
         from ar_lm_decoding_b200 import abi
         self.abi = abi
@@ -192,12 +199,23 @@ class Step:
         self.layer_bytes.append((tail0, off[0]))
         for t in self.q + self.kn + self.vn:
             t.copy_(randn(*t.shape))
-        for t in (self.p_logits, self.q_logits, self.g_logits):
-            t.copy_(randn(*t.shape, std=cfg.sigma, dtype=ldt))
-        self.drafts.copy_(torch.randint(0, V, (B, k), generator=g, device=device, dtype=torch.int32))
-        for t in (self.u_acc, self.u_draft, self.u_res):
-            t.copy_(torch.rand(t.shape, generator=g, device=device))
-        self.pre.zero_()
+        # logits, drafts, pre-accepted flags and uniforms: the seeded recipe the parity tests use (planted peaks
+        # where the workload has them, so that the accept length and the commit's copies vary)
+        vin = synth.make_verify_inputs(cfg, seed=seed)
+
+        def put(dst, a):
+            a = np.ascontiguousarray(a)
+            src = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+            dst.view(src.dtype).copy_(src.reshape(dst.shape))
+
+        put(self.p_logits, vin["p_logits"])
+        put(self.q_logits, vin["q_logits"])
+        put(self.g_logits, vin["group_logits"])
+        put(self.drafts, vin["drafts"])
+        put(self.u_acc, vin["u_acc"])
+        put(self.u_draft, vin["u_draft"])
+        put(self.u_res, vin["u_res"])
+        put(self.pre, vin["preaccepted"])
         self.pre_u8 = self.pre
         # KV caches: one per layer (distinct memory)
         self.kc = [randn(B, Hkv, Pm, D) for _ in range(L)]
@@ -307,17 +325,51 @@ def kernels_per_step(cfg):
     return cfg.L + 2 + 1
 
 
-def gpu_arm(args, cfg):
+def init_ranks(backend):
+    """(world, rank, local rank) from the launcher's environment; joins the process group when world > 1
+    (NCCL for the GPU arm: only the barrier and the max-over-ranks reduction use it)."""
     import torch
     import torch.distributed as dist
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120), **kw)
+    return world, rank, local
+
+
+def replica_dry_run(args, cfg):
+    """The replica bookkeeping alone, on CPU over gloo: every rank joins, passes the barriers, contributes a
+    per-rank time to the max-over-ranks reduction, and rank 0 prints the line's replica fields.  No GPU work:
+    it checks the launcher and the rank plumbing the GPU arm uses."""
+    import torch
+    import torch.distributed as dist
+    world, rank, _ = init_ranks("gloo")
+    ranks = Ranks(world, torch.device("cpu"))
+    ranks.barrier()
+    step_s = ranks.max(1e-3 * (1 + rank))  # rank r pretends a step takes (r+1) ms: the slowest rank counts
+    ranks.barrier()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {"mode": "replica_dry_run", "metric": METRIC, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 5),
+            "value": round(job_throughput(world, step_s), 3), "scaling": "weak",
+            "config": {"workload": workload_desc(cfg, cfg.B),
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}}
+
+
+def gpu_arm(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = init_ranks("nccl")
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
 
@@ -338,8 +390,9 @@ def gpu_arm(args, cfg):
         step.run(stream.cuda_stream)
     torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        graph.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -360,6 +413,7 @@ def gpu_arm(args, cfg):
     ms = max_over_ranks(ms)
     ms_step = ms / args.steps
     assert step.status.item() == 0
+    accept = step.accept_len.cpu().numpy()
 
     # dominant-kernel timing: the step's L tidar_attn_step launches captured alone in a graph on the same
     # stream, replayed and timed with events on that stream (average launch duration as it runs in the step)
@@ -381,52 +435,13 @@ def gpu_arm(args, cfg):
     attn_ms_launch = max_over_ranks(a0.elapsed_time(a1) / (reps * cfg.L))
     del attn_graph
 
-    # e2e: every step copies its inputs from pinned host memory and reads its results back.  The copies run
-    # on a second stream, layer by layer, so that layer l's inputs cross PCIe while layer l-1 computes; each
-    # attention launch waits for its own layer's copy, the verify and commit for theirs, and the result read
-    # closes the step.  One graph holds the whole step; the host waits for it every step.
-    pin_in = torch.empty(step.in_bytes, dtype=torch.uint8, pin_memory=True)
-    pin_in.copy_(step.inbuf[:step.in_bytes])
-    pin_out = torch.empty(step.out_bytes, dtype=torch.uint8, pin_memory=True)
-    copy_stream = torch.cuda.Stream(device)
-    evs = [torch.cuda.Event() for _ in step.layer_bytes]
-    fork = torch.cuda.Event()
-    e2e_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(e2e_graph, stream=stream):
-        fork.record(stream)
-        copy_stream.wait_event(fork)
-        with torch.cuda.stream(copy_stream):
-            for (a, b), ev in zip(step.layer_bytes, evs):
-                step.inbuf[a:b].copy_(pin_in[a:b], non_blocking=True)
-                ev.record(copy_stream)
-        step.prefix.copy_(step.prefix0)
-        for l in range(cfg.L):
-            stream.wait_event(evs[l])
-            step.attn(l, stream.cuda_stream)
-        stream.wait_event(evs[-1])
-        step.verify(stream.cuda_stream)
-        step.commit(stream.cuda_stream)
-        pin_out.copy_(step.outbuf[:step.out_bytes], non_blocking=True)
-    torch.cuda.synchronize()
-    e2e_steps = max(3, min(args.steps, 200))
-    for _ in range(3):
-        e2e_graph.replay()
-    torch.cuda.synchronize()
-    barrier()
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        e2e_graph.replay()
-        stream.synchronize()
-    e2e_s = max_over_ranks(time.perf_counter() - t0)
-    assert int(pin_out[:4].view(torch.int32).item()) >= 0  # the step's accept length, read on the host
-    del e2e_graph
+    e2e = e2e_leg(step, stream, args, barrier, max_over_ranks, world)
 
     del graph
     torch.cuda.synchronize()
 
     peaks, peak_kind = load_peaks()
     hbm = float(peaks["hbm_gbs"])
-    accept = step.accept_len.cpu().numpy()
     byts = algorithmic_bytes(cfg, step.prefix_sum)
     commit_bytes = 4 * cfg.L * cfg.Hkv * cfg.D * int(accept.sum()) * 1  # read new rows + write cache rows (K and V)
     total_bytes = byts["kv"] + byts["qkvo"] + byts["logits"] + commit_bytes
@@ -449,7 +464,8 @@ def gpu_arm(args, cfg):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded, generated on device)",
+        "data": "synthetic (seeded; Q/K/V and caches generated on the device, logits/drafts/uniforms by the "
+                "parity tests' numpy recipe)",
         "config": {"workload": workload_desc(cfg, cfg.B), "batch": cfg.B,
                    "l2": "inputs larger than L2: every layer has its own KV cache "
                          f"({byts['kv'] / 1e6:.0f} MB KV per step vs 126 MB L2)",
@@ -463,18 +479,80 @@ def gpu_arm(args, cfg):
                      "frac": round(achieved / hbm, 4), "traffic": traffic,
                      "kernel": "attn_sm100_kernel (tidar_attn_step: one layer, split-KV merged in-kernel)",
                      "bytes_per_launch": attn_bytes_launch, "us_per_launch": round(attn_ms_launch * 1e3, 3),
+                     "tensor_frac": round(flops / cfg.L / (attn_ms_launch / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
+                                          4),
                      "peak_kind": peak_kind},
         "clocks": ck,
-        "e2e": {"value": round(world * e2e_steps / e2e_s, 3), "unit": UNIT,
-                "h2d_bytes_per_step": step.in_bytes, "d2h_bytes_per_step": step.out_bytes},
+        "e2e": e2e,
         "gpu_launches": kernels_per_step(cfg) * args.steps,
         "accept_len": accept.tolist(),
     }
+    check_line(res)
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_seconds)
     if world > 1:
         dist.destroy_process_group()
     return res if rank == 0 else None
+
+
+def e2e_step(step, stream, copy_stream, events, pin_in, pin_out):
+    """One decode step through the C ABI as a user runs it: this step's inputs (every layer's Q / K_new /
+    V_new, the p / q / group logits, drafts and uniforms) copied from pinned host memory, the L + 2 library
+    calls, the results copied back and read on the host.  The input copies are issued layer by layer on a
+    second stream, so that layer l's inputs cross the host link while layer l-1 computes; every attention call
+    waits only for its own layer's inputs."""
+    import torch
+    cfg = step.cfg
+    copy_stream.wait_stream(stream)  # the previous step no longer reads the input buffer
+    with torch.cuda.stream(copy_stream):
+        for (a, b), ev in zip(step.layer_bytes, events):
+            step.inbuf[a:b].copy_(pin_in[a:b], non_blocking=True)
+            ev.record(copy_stream)
+    with torch.cuda.stream(stream):
+        step.prefix.copy_(step.prefix0)
+        for l in range(cfg.L):
+            stream.wait_event(events[l])
+            step.attn(l, stream.cuda_stream)
+        stream.wait_event(events[-1])
+        step.verify(stream.cuda_stream)
+        step.commit(stream.cuda_stream)
+        pin_out.copy_(step.outbuf[:step.out_bytes], non_blocking=True)
+    stream.synchronize()
+    return int(pin_out[:4].view(torch.int32).item())  # the accept length of sequence 0, read on the host
+
+
+def e2e_leg(step, stream, args, barrier, max_over_ranks, world):
+    """End-to-end steps/s through the public API with host buffers (host wall clock over the timed steps,
+    the host waiting for each step's results; the slowest rank's time)."""
+    import torch
+    pin_in = torch.empty(step.in_bytes, dtype=torch.uint8, pin_memory=True)
+    pin_in.copy_(step.inbuf[:step.in_bytes])
+    pin_out = torch.empty(step.out_bytes, dtype=torch.uint8, pin_memory=True)
+    copy_stream = torch.cuda.Stream(step.dev)
+    events = [torch.cuda.Event() for _ in step.layer_bytes]
+    n = max(3, min(args.steps, 200))
+    for _ in range(3):
+        e2e_step(step, stream, copy_stream, events, pin_in, pin_out)
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        acc = e2e_step(step, stream, copy_stream, events, pin_in, pin_out)
+        assert 0 <= acc <= step.cfg.k
+    s = max_over_ranks(time.perf_counter() - t0)
+    torch.cuda.synchronize()
+    assert step.status.item() == 0
+    return {"value": round(world * n / s, 3), "unit": UNIT, "h2d_bytes_per_step": step.in_bytes,
+            "d2h_bytes_per_step": step.out_bytes, "steps": n,
+            "host_link_gbs": round(step.in_bytes * n / s / 1e9, 2)}
+
+
+def check_line(res):
+    """Sanity rules of the printed line: the end-to-end rate, which adds host copies to the same kernels,
+    cannot exceed the device-timed rate; the dominant kernel cannot take longer than the step."""
+    assert res["e2e"]["value"] <= res["value"] * 1.02, (res["e2e"]["value"], res["value"])
+    us_attn = res["roofline"]["us_per_launch"]
+    assert us_attn * (res["gpu_launches"] / res["steps"] - 3) <= res["ms_per_step"] * 1e3 * 1.05, res
 
 
 def load_traffic(cfg):
@@ -521,6 +599,7 @@ class OracleWorkload:
         self.kn = np.zeros((1, cfg.B, cfg.R, cfg.Hkv, cfg.D), np.uint16)
         self.rng = np.random.default_rng(seed)
         self.cores = oracle.default_threads()
+        self.threads = self.cores
         self.rows_total = cfg.B * cfg.Hq * cfg.R
 
     def attn_rows(self, rows):
@@ -529,14 +608,21 @@ class OracleWorkload:
         sh = self.rng.integers(0, c.Hq, rows)
         sr = self.rng.integers(0, c.R, rows)
         t0 = time.perf_counter()
-        self.oracle.attn_rows(self.inp, c.Hq, c.Hkv, c.D, c.k, sb, sh, sr)
+        self.oracle.attn_rows(self.inp, c.Hq, c.Hkv, c.D, c.k, sb, sh, sr, nthreads=self.threads)
+        return time.perf_counter() - t0
+
+    def attn_layer(self):
+        """All query rows of one layer (every sequence, head and row)."""
+        c = self.cfg
+        t0 = time.perf_counter()
+        self.oracle.attn(self.inp, c.Hq, c.Hkv, c.D, c.k, dense=False, nthreads=self.threads)
         return time.perf_counter() - t0
 
     def verify_commit(self):
         t0 = time.perf_counter()
-        out = self.oracle.verify(self.v)
+        out = self.oracle.verify(self.v, nthreads=self.threads)
         self.oracle.kv_commit(self.kc, self.kc, self.kn, self.kn, self.inp["prefix_len"], out["accept_len"],
-                              out["resampled"], self.v["group_logits"], self.v["u_draft"])
+                              out["resampled"], self.v["group_logits"], self.v["u_draft"], nthreads=self.threads)
         return time.perf_counter() - t0
 
     def rows_for(self, seconds):
@@ -545,38 +631,65 @@ class OracleWorkload:
         return int(min(self.rows_total, max(1, seconds / max(per_row, 1e-7))))
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def host_cores():
+    return {"affinity": len(os.sched_getaffinity(0)), "nproc": os.cpu_count(), "cpu_model": cpu_model()}
+
+
 def cpu_baseline(cfg, seconds):
-    """Oracle steps/s on the host cores from a bounded sample of attention rows."""
+    """Oracle steps/s on the host cores from a bounded sample of attention rows, with OpenMP over all the
+    cores this process may use and single-threaded."""
     w = OracleWorkload(cfg)
-    rows = max(w.cores, w.rows_for(seconds))
-    t_rows, reps = 0.0, 0
-    while reps < 1 or (t_rows < seconds and reps < 50):  # repeat a whole-layer sample up to ~`seconds`
-        t_rows += w.attn_rows(rows)
-        reps += 1
-    t_rows /= reps
-    t_vc = w.verify_commit()
-    t_step = cfg.L * t_rows * w.rows_total / rows + t_vc
-    return {"value": round(1.0 / t_step, 6), "unit": UNIT, "cores": w.cores, "kind": "oracle",
-            "sample": f"{rows} of {w.rows_total} attention rows of one layer, timed {reps}x (scaled "
-                      f"x{w.rows_total / rows:.1f} and x{cfg.L} layers, which do identical work), plus the full "
-                      f"verify and commit with draft selection; {reps * t_rows + t_vc:.1f} s of wall time on "
-                      f"{w.cores} threads",
-            "seconds_per_step": round(t_step, 3)}
+    res = {}
+    for label, threads, budget in (("all_cores", w.cores, seconds), ("single_thread", 1, seconds / 3)):
+        w.threads = threads
+        rows = max(threads, w.rows_for(budget))
+        t_rows, reps = 0.0, 0
+        while reps < 1 or (t_rows < budget and reps < 50):  # repeat the row sample up to ~`budget` seconds
+            t_rows += w.attn_rows(rows)
+            reps += 1
+        t_rows /= reps
+        t_vc = w.verify_commit()
+        t_step = cfg.L * t_rows * w.rows_total / rows + t_vc
+        res[label] = {"value": round(1.0 / t_step, 6), "threads": threads, "seconds_per_step": round(t_step, 3),
+                      "sample": f"{rows} of {w.rows_total} attention rows of one layer, timed {reps}x (scaled "
+                                f"x{w.rows_total / rows:.1f} and x{cfg.L} layers, which do identical work), plus "
+                                f"the full verify and commit with draft selection; {reps * t_rows + t_vc:.1f} s "
+                                f"of wall time"}
+    a = res["all_cores"]
+    return {"value": a["value"], "unit": UNIT, "cores": a["threads"], "kind": "oracle", "sample": a["sample"],
+            "seconds_per_step": a["seconds_per_step"], "single_thread": res["single_thread"], "host": host_cores()}
 
 
 def reference_arm(args, cfg):
-    """The oracle as the reference implementation: each step times a bounded sample of the workload."""
+    """The oracle as the reference implementation.  Every timed step is a whole decode step of the workload:
+    the oracle's attention over all query rows of a layer, run once per layer (the same layer inputs L times:
+    the layers do identical work), then its verify and its commit with draft selection.  The warm-up steps
+    run one layer each (untimed)."""
     w = OracleWorkload(cfg)
-    budget = 90.0  # seconds for all attention samples of the run
-    rows = max(1, w.rows_for(budget / (args.steps + args.warmup)))
-    t_vc = min(w.verify_commit() for _ in range(3))  # timed three times outside the steps, best taken
     for _ in range(args.warmup):
-        w.attn_rows(rows)
-    tot = sum(w.attn_rows(rows) for _ in range(args.steps))
-    t_step = cfg.L * (tot / args.steps) * w.rows_total / rows + t_vc
+        w.attn_layer()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(cfg.L):
+            w.attn_layer()
+        w.verify_commit()
+    t_step = (time.perf_counter() - t0) / args.steps
     value = 1.0 / t_step
-    sample = (f"each step: {rows} of {w.rows_total} attention rows of one layer, scaled to the layer and to "
-              f"{cfg.L} layers; the verify and commit (full) timed separately and added")
+    sample = (f"each timed step: all {w.rows_total} attention rows of a layer x {cfg.L} layers (the same layer "
+              f"inputs each time), then the full verify and commit with draft selection, on {w.cores} threads; "
+              f"warm-up steps run one layer")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 3),
@@ -584,7 +697,7 @@ def reference_arm(args, cfg):
         "data": "synthetic (seeded numpy)",
         "config": {"workload": workload_desc(cfg, cfg.B), "batch": cfg.B},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": w.cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_cores()},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -633,7 +746,21 @@ def attn_prefix_sweep(args, cfg):
                       "us_per_key_tile": round(slope, 4)}), flush=True)
 
 
-def main():
+def replica_command(argv, n, port):
+    """The torchrun command that runs this script as `n` replicas on one node (one process per GPU)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", str(n),
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5000)
@@ -644,25 +771,36 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-prefix-sweep", action="store_true",
                     help="print attention time per launch against the prefix length (not the benchmark line)")
-    args = ap.parse_args()
+    ap.add_argument("--replica-dry-run", action="store_true",
+                    help="run only the replica bookkeeping on CPU (gloo) and print its fields (no GPU work)")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
     from ar_lm_decoding_b200 import synth
     cfg = synth.CONFIGS[args.config]
+    world = os.environ.get("WORLD_SIZE")
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
-            return
+            return 0
         import oracle
         oracle.build()
         print(json.dumps(reference_arm(args, cfg)), flush=True)
-        return
+        return 0
     if args.attn_prefix_sweep:
         attn_prefix_sweep(args, cfg)
-        return
-    res = gpu_arm(args, cfg)
+        return 0
+    if world is None and args.gpus > 1:
+        # not under a launcher: start the N replicas (one process per GPU) and pass on their exit status
+        return subprocess.call(replica_command(argv, args.gpus, free_port()))
+    if world is not None and int(world) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started {world} processes")
+    res = replica_dry_run(args, cfg) if args.replica_dry_run else gpu_arm(args, cfg)
     if res is not None:
         print(json.dumps(res), flush=True)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

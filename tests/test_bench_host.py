@@ -81,3 +81,22 @@ def test_reference_arm_line():
     assert res["e2e"] == {"value": res["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                           "d2h_bytes_per_step": 0}
     json.dumps(res)
+
+
+def test_line_sanity_rules():
+    line = {"value": 1000.0, "ms_per_step": 1.0, "steps": 10, "gpu_launches": 390,
+            "roofline": {"us_per_launch": 20.0}, "e2e": {"value": 500.0}}
+    bench.check_line(line)
+    with pytest.raises(AssertionError):  # end to end cannot beat the device-only rate
+        bench.check_line({**line, "e2e": {"value": 1500.0}})
+    with pytest.raises(AssertionError):  # 36 attention launches of 30 us do not fit a 1 ms step
+        bench.check_line({**line, "roofline": {"us_per_launch": 30.0}})
+
+
+def test_cpu_baseline_reports_single_thread_and_all_cores():
+    import oracle
+    oracle.build()
+    cb = bench.cpu_baseline(synth.CONFIGS["tiny"], 0.2)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert cb["single_thread"]["threads"] == 1 and cb["single_thread"]["value"] > 0
+    assert cb["host"]["nproc"] >= 1 and cb["host"]["cpu_model"]
