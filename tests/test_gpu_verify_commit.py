@@ -13,45 +13,15 @@ import pytest
 
 import oracle
 from ar_lm_decoding_b200 import synth
+from parity import compare_next_drafts, compare_verify
 
 pytestmark = pytest.mark.gpu
 
-EXEMPT = 1e-5
 
 
 def _gpu():
     import tidar_gpu
     return tidar_gpu
-
-
-def _compare_verify(inp, got, report):
-    ref = oracle.verify(inp)
-    B, k = inp["drafts"].shape
-    forced = np.full(B, -1, np.int32)
-    for b in range(B):
-        if got["accept_len"][b] != ref["accept_len"][b]:
-            i = min(got["accept_len"][b], ref["accept_len"][b])  # first slot decided differently
-            margin = abs(float(inp["u_acc"][b, i]) - ref["ratio"][b, i])
-            assert margin < EXEMPT, (b, got["accept_len"][b], ref["accept_len"][b], margin)
-            report.append(("accept", b, margin))
-            forced[b] = got["accept_len"][b]
-    if (forced >= 0).any():
-        ref = oracle.verify(inp, forced_accept_len=forced)
-    assert np.array_equal(got["accept_len"], ref["accept_len"])
-    for b in range(B):
-        if got["resampled"][b] != ref["resampled"][b]:
-            u = float(inp["u_res"][b])
-            margin = min(abs(u - ref["res_lo"][b]), abs(u - ref["res_hi"][b]))
-            assert margin < EXEMPT, (b, got["resampled"][b], ref["resampled"][b], margin)
-            report.append(("resample", b, margin))
-            ref["resampled"][b] = got["resampled"][b]
-            ref["tokens"][b, ref["n_emitted"][b] - 1] = got["resampled"][b]
-    assert np.array_equal(got["resampled"], ref["resampled"])
-    assert np.array_equal(got["n_emitted"], ref["n_emitted"])
-    assert np.array_equal(got["tokens"], ref["tokens"])
-    np.testing.assert_allclose(got["logp_d"], ref["logp_d"], rtol=0, atol=1e-4)
-    np.testing.assert_allclose(got["logq_d"], ref["logq_d"], rtol=0, atol=1e-4)
-    return ref
 
 
 @pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k4", "qwen2.5-1.5b_k16", "qwen3-8b_k8", "qwen3-8b_k8_b8",
@@ -62,7 +32,7 @@ def test_verify_parity(name):
     for seed in range(3):
         inp = synth.make_verify_inputs(cfg, seed=seed)
         got = _gpu().verify(inp)
-        _compare_verify(inp, got, report)
+        compare_verify(inp, got, report)
     print(f"{name}: exemptions {report}")
     assert len(report) <= 1
 
@@ -81,7 +51,7 @@ def test_verify_many_small_cases():
         zq[: B // 2] = zp[: B // 2] + 0.1 * rng.standard_normal(zp[: B // 2].shape).astype(np.float32)
         inp["q_logits"] = synth.f32_to_bf16_bits(zq) if dtype == "bf16" else zq
         got = _gpu().verify(inp)
-        _compare_verify(inp, got, report)
+        compare_verify(inp, got, report)
         assert len(set(got["accept_len"].tolist())) > 1
     print(f"exemptions {report}")
     assert len(report) <= 2
@@ -126,12 +96,7 @@ def test_commit_parity(name):
         assert np.array_equal(got["prefix_len"], ref["prefix_len"])
         assert np.array_equal(got["next_q_group"], ref["next_q_group"])
         assert np.array_equal(got["next_preaccepted"], ref["next_preaccepted"])
-        diff = got["next_drafts"] != ref["next_drafts"]
-        for b, s in zip(*np.nonzero(diff)):
-            u = float(ud[b, s])
-            margin = min(abs(u - ref["draft_lo"][b, s]), abs(u - ref["draft_hi"][b, s]))
-            assert margin < EXEMPT, (b, s, got["next_drafts"][b, s], ref["next_drafts"][b, s], margin)
-            report.append(("draft", b, s, margin))
+        compare_next_drafts(got, ref, ud, report)
     print(f"{name}: exemptions {report}")
     assert len(report) <= 1
 
@@ -155,7 +120,7 @@ def test_step_chain_state_machine():
     cfg = synth.CONFIGS["qwen2.5-1.5b_k4"].with_(B=4, V=30000, ragged=(100, 400))
     inp = synth.make_verify_inputs(cfg, seed=9)
     got = _gpu().verify(inp)
-    ref = _compare_verify(inp, got, [])
+    ref = compare_verify(inp, got, [])
     kc, vc, kn, vn, pl, _, _, g, ud = _commit_inputs(cfg, 9, L=2)
     cg = _gpu().kv_commit(kc, vc, kn, vn, pl, got["accept_len"], got["resampled"], inp["group_logits"],
                           inp["u_draft"])
