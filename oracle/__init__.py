@@ -107,7 +107,9 @@ def _logits_arg(a):
     return np.ascontiguousarray(a, dtype=np.float32), LOGITS_F32
 
 
-def verify(inp: dict, forced_accept_len=None, nthreads: int = 0) -> dict:
+def verify(inp: dict, forced_accept_len=None, nthreads: int = 0, trust_ar: float = 1.0) -> dict:
+    """AR rejection-sampling verify; trust_ar = lambda mixes the target logits as
+    lambda * p_logits + (1 - lambda) * q_logits (1: the AR logits alone)."""
     p, dt = _logits_arg(inp["p_logits"])
     q, dt2 = _logits_arg(inp["q_logits"])
     assert dt == dt2
@@ -122,7 +124,7 @@ def verify(inp: dict, forced_accept_len=None, nthreads: int = 0) -> dict:
         n_emitted=np.zeros(B, np.int32), logp_d=np.zeros((B, k)), logq_d=np.zeros((B, k)), ratio=np.zeros((B, k)),
         res_lo=np.zeros(B), res_hi=np.zeros(B))
     rc = lib().oracle_verify(_p(p), _p(q), ctypes.c_int(dt), _p(drafts), _p(pre), _p(ua), _p(ur),
-                             ctypes.c_int(B), ctypes.c_int(k), ctypes.c_int(V), _p(forced),
+                             ctypes.c_int(B), ctypes.c_int(k), ctypes.c_int(V), ctypes.c_double(trust_ar), _p(forced),
                              ctypes.c_int(nthreads or default_threads()),
                              *[_p(out[n]) for n in ("accept_len", "resampled", "tokens", "n_emitted", "logp_d",
                                                     "logq_d", "ratio", "res_lo", "res_hi")])

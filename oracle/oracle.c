@@ -252,6 +252,41 @@ static double log_prob(const void *base, int dtype, size_t off, row_stats st, in
 }
 
 /*
+ * The verify's target logits: lambda * z_AR + (1 - lambda) * z_diff ("Trust AR
+ * vs trust diffusion logits", Fig. 6 of the summary: the AR and diffusion
+ * logits are mixed with a weight lambda at verification).  lambda = 1 is the
+ * AR row itself, lambda = 0 the diffusion row itself (taken as stored, so that
+ * an infinite logit never meets a zero weight).
+ */
+typedef struct {
+    const void *p, *q;
+    int dtype;
+    size_t off_p, off_q;
+    double lambda;
+} target_row;
+
+static double target_logit(const target_row *t, int v) {
+    if (t->lambda == 1.0) return logit_value(t->p, t->dtype, t->off_p + v);
+    if (t->lambda == 0.0) return logit_value(t->q, t->dtype, t->off_q + v);
+    return t->lambda * logit_value(t->p, t->dtype, t->off_p + v) +
+           (1.0 - t->lambda) * logit_value(t->q, t->dtype, t->off_q + v);
+}
+
+static row_stats target_stats(const target_row *t, int V) {
+    row_stats st = {-INFINITY, 0.0};
+    for (int v = 0; v < V; ++v) {
+        const double z = target_logit(t, v);
+        if (z > st.m) st.m = z;
+    }
+    for (int v = 0; v < V; ++v) st.Z += exp(target_logit(t, v) - st.m);
+    return st;
+}
+
+static double target_log_prob(const target_row *t, row_stats st, int v) {
+    return target_logit(t, v) - st.m - log(st.Z);
+}
+
+/*
  * Smallest token t whose inclusive cumulative weight exceeds u * total, for
  * non-negative weights w(v).  Reports the chosen token's interval of the
  * normalised CDF in [lo, hi).  Returns -1 if the total weight is zero.
@@ -285,23 +320,21 @@ static int inverse_cdf(weight_fn w, const void *ctx, int V, double u, double *lo
 }
 
 typedef struct {
-    const void *p, *q;
-    int dtype;
-    size_t off_p, off_q;
+    target_row t;
     row_stats sp, sq;
 } residual_ctx;
 
-/* max(0, p(v) - q(v)): the residual distribution of a rejected draft. */
+/* max(0, p(v) - q(v)): the residual distribution of a rejected draft (p the verify's target). */
 static double residual_weight(const void *c, int v) {
     const residual_ctx *r = (const residual_ctx *)c;
-    const double pv = exp(log_prob(r->p, r->dtype, r->off_p, r->sp, v));
-    const double qv = exp(log_prob(r->q, r->dtype, r->off_q, r->sq, v));
+    const double pv = exp(target_log_prob(&r->t, r->sp, v));
+    const double qv = exp(log_prob(r->t.q, r->t.dtype, r->t.off_q, r->sq, v));
     return pv > qv ? pv - qv : 0.0;
 }
 
 static double p_weight(const void *c, int v) {
     const residual_ctx *r = (const residual_ctx *)c;
-    return exp(log_prob(r->p, r->dtype, r->off_p, r->sp, v));
+    return exp(target_log_prob(&r->t, r->sp, v));
 }
 
 typedef struct {
@@ -326,14 +359,16 @@ static double softmax_weight(const void *c, int v) {
  * slot.  A pre-accepted slot 1 (the previous step's resampled token) is
  * accepted unconditionally.  Slot 1's p is the AR row carried from the
  * previous forward; slot i > 1 uses the causal logits of draft row i-1.
+ * With trust_ar = lambda < 1 the target p is softmax of the mixed logits
+ * lambda * z_AR + (1 - lambda) * z_diff (see target_logit).
  */
 int oracle_verify(const void *p_logits, const void *q_logits, int logits_dtype,
                   const int32_t *drafts, const uint8_t *preaccepted,
-                  const float *u_acc, const float *u_res, int B, int k, int V,
+                  const float *u_acc, const float *u_res, int B, int k, int V, double trust_ar,
                   const int32_t *forced_accept_len, int nthreads,
                   int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
                   double *logp_d, double *logq_d, double *ratio, double *res_lo, double *res_hi) {
-    if (B < 1 || k < 1 || V < 1) return 1;
+    if (B < 1 || k < 1 || V < 1 || !(trust_ar >= 0.0 && trust_ar <= 1.0)) return 1;
     for (size_t i = 0; i < (size_t)B * k; ++i)
         if (drafts[i] < 0 || drafts[i] >= V) return 1;
     set_threads(nthreads);
@@ -342,9 +377,10 @@ int oracle_verify(const void *p_logits, const void *q_logits, int logits_dtype,
 #pragma omp parallel for schedule(dynamic, 1)
     for (long t = 0; t < 2L * B * k; ++t) {
         const long row = t / 2;
-        if (t % 2 == 0)
-            sp[row] = softmax_stats(p_logits, logits_dtype, (size_t)row * V, V);
-        else
+        if (t % 2 == 0) {
+            const target_row tr = {p_logits, q_logits, logits_dtype, (size_t)row * V, (size_t)row * V, trust_ar};
+            sp[row] = target_stats(&tr, V);
+        } else
             sq[row] = softmax_stats(q_logits, logits_dtype, (size_t)row * V, V);
     }
 #pragma omp parallel for schedule(dynamic, 1)
@@ -354,7 +390,8 @@ int oracle_verify(const void *p_logits, const void *q_logits, int logits_dtype,
         for (int i = 0; i < k; ++i) {
             const size_t row = (size_t)b * k + i;
             const int d = drafts[row];
-            logp_d[row] = log_prob(p_logits, logits_dtype, row * V, sp[row], d);
+            const target_row tr = {p_logits, q_logits, logits_dtype, row * V, row * V, trust_ar};
+            logp_d[row] = target_log_prob(&tr, sp[row], d);
             logq_d[row] = log_prob(q_logits, logits_dtype, row * V, sq[row], d);
             ratio[row] = NAN;
             if (stopped) continue;
@@ -377,7 +414,7 @@ int oracle_verify(const void *p_logits, const void *q_logits, int logits_dtype,
         resampled[b] = -1;
         if (j < k) {
             const size_t row = (size_t)b * k + j;
-            residual_ctx rc = {p_logits, q_logits, logits_dtype, row * V, row * V, sp[row], sq[row]};
+            residual_ctx rc = {{p_logits, q_logits, logits_dtype, row * V, row * V, trust_ar}, sp[row], sq[row]};
             double lo = NAN, hi = NAN;
             int t = inverse_cdf(residual_weight, &rc, V, (double)u_res[b], &lo, &hi);
             if (t < 0) t = inverse_cdf(p_weight, &rc, V, (double)u_res[b], &lo, &hi); /* p == q */

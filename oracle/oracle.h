@@ -53,7 +53,9 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k_new, const uint16_t *v
                      int nthreads, double *o, double *lse);
 
 /* AR rejection-sampling verify.  p/q logits: [B,k,V]; drafts [B,k];
- * preaccepted [B]; u_acc [B,k]; u_res [B].  forced_accept_len (nullable,
+ * preaccepted [B]; u_acc [B,k]; u_res [B].  trust_ar in [0, 1]: the target
+ * distribution is softmax(trust_ar * p_logits + (1 - trust_ar) * q_logits)
+ * (1 = the AR logits alone).  forced_accept_len (nullable,
  * entries < 0 mean "not forced") overrides the accept decision (used to keep
  * comparing after an exempt near-tie).  Outputs: accept_len [B], resampled [B]
  * (-1 if every draft was accepted), tokens [B,k] (-1 padded), n_emitted [B],
@@ -62,7 +64,7 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k_new, const uint16_t *v
  * CDF; NaN when no resample). */
 int oracle_verify(const void *p_logits, const void *q_logits, int logits_dtype,
                   const int32_t *drafts, const uint8_t *preaccepted,
-                  const float *u_acc, const float *u_res, int B, int k, int V,
+                  const float *u_acc, const float *u_res, int B, int k, int V, double trust_ar,
                   const int32_t *forced_accept_len, int nthreads,
                   int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
                   double *logp_d, double *logq_d, double *ratio, double *res_lo, double *res_hi);

@@ -266,3 +266,60 @@ def test_synth_peaks_drive_accept_length():
     m = inp["m_shared"]
     pre = inp["preaccepted"].astype(np.int32)
     assert np.abs(out["accept_len"] - np.maximum(m, pre)).max() <= 1
+
+
+# ---- trust-mix verify (lambda mixes the AR and diffusion logits of the target) ----
+
+
+def test_trust_mix_hand_worked_example():
+    p = np.log(np.array([0.5, 0.3, 0.2]))
+    q = np.log(np.array([0.2, 0.3, 0.5]))
+    for d, ua, ur, acc, res, ratio, lo, hi in read_golden("verify_trust_mix_hand.txt"):
+        inp = _verify_inputs(p[None, None], q[None, None], [[int(d)]], [[float(ua)]], [float(ur)])
+        out = oracle.verify(inp, trust_ar=0.5)
+        assert out["accept_len"][0] == int(acc) and out["resampled"][0] == int(res), (d, ua, ur)
+        assert abs(out["ratio"][0, 0] - float(ratio)) < 2e-6
+        if lo == "nan":
+            assert np.isnan(out["res_lo"][0])
+        else:
+            assert abs(out["res_lo"][0] - float(lo)) < 2e-6 and abs(out["res_hi"][0] - float(hi)) < 2e-6
+
+
+def test_trust_mix_endpoints():
+    rng = np.random.default_rng(4)
+    B, k, V = 40, 4, 30
+    zp = (rng.standard_normal((B, k, V)) * 2).astype(np.float32)
+    zq = (rng.standard_normal((B, k, V)) * 2).astype(np.float32)
+    inp = _verify_inputs(zp, zq, rng.integers(0, V, (B, k)), rng.random((B, k)), rng.random(B))
+    # lambda = 1: the plain AR verify
+    a, b = oracle.verify(inp), oracle.verify(inp, trust_ar=1.0)
+    for n in ("accept_len", "resampled", "tokens", "n_emitted"):
+        assert np.array_equal(a[n], b[n])
+    # lambda = 0: the target is q itself, every draft has ratio 1 and is accepted
+    z = oracle.verify(inp, trust_ar=0.0)
+    assert (z["accept_len"] == k).all() and (z["resampled"] == -1).all()
+    assert np.allclose(z["logp_d"], z["logq_d"])
+    with pytest.raises(ValueError):
+        oracle.verify(inp, trust_ar=1.5)
+
+
+def test_trust_mix_is_lossless_for_its_target():
+    """With d ~ q, the first emitted token is distributed as p_lambda = softmax(lambda z_p + (1 - lambda) z_q)
+    (speculative sampling is exact for whatever target it verifies against)."""
+    lam, V, trials = 0.3, 8, 200000
+    rng, P_, Q_ = _mc_setup(V, seed=77, k=1)
+    zp, zq = np.log(P_[0]).astype(np.float32), np.log(Q_[0]).astype(np.float32)
+    counts = np.zeros(V)
+    for start in range(0, trials, 20000):
+        B = 20000
+        drafts = rng.choice(V, size=(B, 1), p=np.exp(zq.astype(np.float64)) / np.exp(zq.astype(np.float64)).sum())
+        inp = _verify_inputs(np.broadcast_to(zp, (B, 1, V)).copy(), np.broadcast_to(zq, (B, 1, V)).copy(), drafts,
+                             rng.random((B, 1)), rng.random(B))
+        out = oracle.verify(inp, trust_ar=lam)
+        counts += np.bincount(out["tokens"][:, 0], minlength=V)
+    target = np.exp(lam * zp.astype(np.float64) + (1 - lam) * zq.astype(np.float64))
+    target /= target.sum()
+    assert stats.chisquare(counts, counts.sum() * target).pvalue > 1e-3
+    # and it is not the AR distribution itself
+    pa = np.exp(zp.astype(np.float64)) / np.exp(zp.astype(np.float64)).sum()
+    assert stats.chisquare(counts, counts.sum() * pa).pvalue < 1e-6
