@@ -159,3 +159,25 @@ def kv_commit(k_caches, v_caches, k_news, v_news, prefix_len, accept_len, resamp
         raise ValueError("oracle_kv_commit: invalid arguments")
     out.update(k_caches=kc, v_caches=vc, prefix_len=pl)
     return out
+
+
+def row_positions(k: int, P: int) -> np.ndarray:
+    """Positions of the R = k(k+2) rows of a step with cached prefix P."""
+    R = k * (k + 2)
+    return np.array([lib().oracle_row_position(ctypes.c_int(k), ctypes.c_int(P), ctypes.c_int(r)) for r in range(R)],
+                    dtype=np.int64)
+
+
+def rope_qkv(qkv, prefix_len, Hq: int, Hkv: int, k: int, theta: float = 1e6):
+    """Rotary embedding of qkv [B,R,Hq+2Hkv,D] (bf16 bits) -> (q, k_new, v_new) bf16 bits."""
+    x = _c(qkv, np.uint16)
+    B, R, H, D = x.shape
+    q = np.zeros((B, R, Hq, D), np.uint16)
+    kn = np.zeros((B, R, Hkv, D), np.uint16)
+    vn = np.zeros((B, R, Hkv, D), np.uint16)
+    pl = _c(prefix_len, np.int32)
+    rc = lib().oracle_rope_qkv(_p(x), _p(pl), ctypes.c_int(B), ctypes.c_int(Hq), ctypes.c_int(Hkv), ctypes.c_int(D),
+                               ctypes.c_int(k), ctypes.c_double(theta), _p(q), _p(kn), _p(vn))
+    if rc:
+        raise ValueError("oracle_rope_qkv: invalid arguments")
+    return q, kn, vn

@@ -493,3 +493,54 @@ int oracle_kv_commit(uint16_t *k_caches, uint16_t *v_caches,
     }
     return 0;
 }
+
+/* ---- rotary position embedding of the step's rows --------------------- */
+/*
+ * Positions of the R = k(k+2) rows of one step (reading of "并行 self-speculative
+ * 生成 (§3.2)" of the summary, where the pages give the partitions but not the
+ * positions): draft d_i (row i-1) continues the prefix at P + i - 1; pre-draft
+ * group j (the continuation after j accepted drafts) puts its slot s at
+ * P + j + s.
+ */
+int oracle_row_position(int k, int P, int r) {
+    if (r < k) return P + r;
+    const int j = (r - k) / k, s = (r - k) % k;
+    return P + j + s;
+}
+
+/*
+ * Rotary embedding with base theta, in the half-split layout of the Qwen
+ * backbones the pages start from: for i < D/2 the pair (x_i, x_{i+D/2}) is
+ * rotated by the angle pos * theta^(-2i/D).  qkv: bf16 [B, R, Hq + 2 Hkv, D]
+ * (the fused projection output: Q heads, then K heads, then V heads); outputs
+ * q [B, R, Hq, D], k_new and v_new [B, R, Hkv, D], bf16 rounded to nearest
+ * even from double.  V is copied.
+ */
+int oracle_rope_qkv(const uint16_t *qkv, const int32_t *prefix_len, int B, int Hq, int Hkv, int D, int k,
+                    double theta, uint16_t *q, uint16_t *k_new, uint16_t *v_new) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || k < 1 || D < 2 || D % 2 || !(theta > 1.0)) return 1;
+    const int R = k * (k + 2), H = Hq + 2 * Hkv, half = D / 2;
+    for (int b = 0; b < B; ++b)
+        for (int r = 0; r < R; ++r) {
+            const double pos = (double)oracle_row_position(k, prefix_len[b], r);
+            for (int h = 0; h < H; ++h) {
+                const uint16_t *x = qkv + (((size_t)b * R + r) * H + h) * D;
+                uint16_t *y;
+                if (h < Hq) y = q + (((size_t)b * R + r) * Hq + h) * D;
+                else if (h < Hq + Hkv) y = k_new + (((size_t)b * R + r) * Hkv + (h - Hq)) * D;
+                else y = v_new + (((size_t)b * R + r) * Hkv + (h - Hq - Hkv)) * D;
+                if (h >= Hq + Hkv) {
+                    for (int d = 0; d < D; ++d) y[d] = x[d];
+                    continue;
+                }
+                for (int i = 0; i < half; ++i) {
+                    const double ang = pos * pow(theta, -2.0 * i / D);
+                    const double c = cos(ang), sn = sin(ang);
+                    const double a = bf16_value(x[i]), bb = bf16_value(x[i + half]);
+                    y[i] = bf16_round(a * c - bb * sn);
+                    y[i + half] = bf16_round(bb * c + a * sn);
+                }
+            }
+        }
+    return 0;
+}

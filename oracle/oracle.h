@@ -83,6 +83,14 @@ int oracle_kv_commit(uint16_t *k_caches, uint16_t *v_caches,
                      int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group,
                      double *draft_lo, double *draft_hi);
 
+/* Position of row r (0..R-1) of a step whose sequence has cached prefix P. */
+int oracle_row_position(int k, int P, int r);
+
+/* Rotary embedding of the fused QKV projection output qkv [B,R,Hq+2Hkv,D]
+ * (bf16 bits) into q [B,R,Hq,D], k_new and v_new [B,R,Hkv,D] (bf16 bits). */
+int oracle_rope_qkv(const uint16_t *qkv, const int32_t *prefix_len, int B, int Hq, int Hkv, int D, int k,
+                    double theta, uint16_t *q, uint16_t *k_new, uint16_t *v_new);
+
 #ifdef __cplusplus
 }
 #endif
