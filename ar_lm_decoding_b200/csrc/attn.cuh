@@ -16,7 +16,16 @@ struct AttnParams {
     bf16 *out;         // [B, R, Hq, D]
     float *lse;        // [B, R, Hq] or null
     int32_t *dev_status;
+    // paged KV cache (null: contiguous [B, Hkv, P_max, D] caches): cache row n of sequence b is row n % 64 of
+    // page block_table[b * max_pages + n / 64] of the pool [num_pages, Hkv, 64, D]; P_max = 64 * max_pages
+    const int32_t *block_table;
+    int max_pages, num_pages;
+    long long wait_cycles;  // bound of every on-chip wait, in SM clock cycles
+    int stall_test;         // 1: the QK issuer first waits on a barrier nothing arrives on (timeout test)
 };
+
+// Bound of the on-chip waits of a normal launch (about 2 s at the B200's clocks).
+constexpr long long kAttnWaitCycles = 4000000000LL;
 
 int attn_sm100_rows_per_tile();
 int attn_sm100_keys_per_tile();

@@ -2,48 +2,59 @@
 //
 // One CTA owns 128 packed query rows (row m = r*G + g of the G query heads
 // sharing KV head kvh: GQA packing, so every K/V byte feeds 128 rows) and a
-// contiguous run of 128-key tiles of one sequence.  A sequence's tiles are
-// the cached prefix in 128-row tiles (the last one partial) followed by the
-// R new keys of this step in 128-row tiles.
+// contiguous run of 64-key tiles of one sequence.  A sequence's tiles are
+// the cached prefix in 64-row tiles (the last one partial) followed by the
+// R new keys of this step in 64-row tiles.
 //
 // Warp roles (12 warps):
 //   warps 0, 2  TMA producers of K and of V (128-byte swizzle), each into its
-//               own 3-stage ring: prefix tiles from the cache, new-key tiles
+//               own 4-stage ring: prefix tiles from the cache, new-key tiles
 //               from K_new/V_new through a 3-D tensor map (no head gather).
 //               A K stage is freed when its QK^T completes, a V stage when
 //               its PV does, so K runs ahead of V.
 //   warp 1      TMEM owner; one thread issues S = Q K^T (tcgen05.mma, both
-//               operands in shared memory) into S buffer j % 3.
-//   warp 3      one thread issues O += P V with P read from TMEM (A operand
+//               operands in shared memory) into S buffer i % 4.
+//   warp 3      one thread issues O_w += P V with P read from TMEM (A operand
 //               in TMEM, V an MN-major operand in shared memory).
-//   warps 4-11  softmax: both warpgroups work on every tile, warpgroup w on
-//               its columns [64w, 64w+64); thread = query row = TMEM lane.
-//               The two halves of a row always hold the same running max,
-//               so their exponentials share a scale and PV sums them into
-//               the one O.  A tile is exponentiated against that (possibly
-//               stale) max -- exact as long as p <= 2^8 fits -- while its row
-//               max is taken in the same pass; the halves then exchange
-//               maxima through shared memory, and only rows whose max grew
-//               by more than 2^8 redo their exponentials and rescale O.  The
-//               mask is evaluated from indices.
-//   warps 2-3   also load Q when its rows cannot come through TMA.
-// TMEM (512 columns): S buffers at [0, 128), [128, 256), [256, 384); O at
-// [384, 384+D).  P (bf16) overwrites the first 64 columns of its S buffer.
-// QK(j) reuses the buffer that PV(j-3) reads and is issued once PV(j-3) has
-// completed, so the softmax always has the next two tiles' S ready.
-// The CTAs that split one row tile's keys form a thread-block cluster.  At the
-// end each warpgroup reads its half of the columns of O from TMEM and forms
-// one normalised partial row per query row, stored as
-// fp16 with a per-half-row fp32 scale (|error| <= 2^-12 of the row maximum)
-// and its log2 LSE in fp32.  With one split that row is the output.  Otherwise
-// the records are pushed over distributed shared memory into the idle K/V ring
-// of the cluster CTA that owns the row (a split cluster barrier: arrive once
-// the ring is idle, wait before pushing); after a second cluster barrier each
-// CTA merges its slice of rows over the S partials (LSE weights, fixed order)
-// and writes the final bf16 output and LSE.
+//   warps 4-11  softmax, two warpgroups that take alternate key tiles:
+//               warpgroup w owns tiles i = w, w+2, w+4, ... of the CTA's run,
+//               S buffers w and w+2 (double buffered: the S of its next tile
+//               is computed while it works on this one) and its own
+//               accumulator O_w.  Thread = query row = TMEM lane, so each
+//               thread holds the whole row of its tile (64 scores in
+//               registers): the row max first, then the exponentials; the
+//               running max only moves (and O_w is rescaled) when the tile
+//               max exceeds it by more than 2^8, so p <= 2^8 always fits.  The
+//               two warpgroups never wait for each other.  The mask is
+//               evaluated from indices.
+//   warps 2-11  also load Q when its rows cannot come through TMA.
+// TMEM (512 columns): S buffers at [64 j, 64 j + 64), j = 0..3; O_0 at
+// [256, 256+D), O_1 at [384, 384+D).  P (bf16) overwrites the first 32
+// columns of its S buffer.  QK(i) reuses the buffer that PV(i-4) reads and is
+// issued once PV(i-4) has completed.
+// At the end the two accumulators of a row are merged with the weights of
+// their running maxima (each warpgroup takes half of the columns), giving one
+// normalised partial row per query row, stored as fp16 with a per-half-row
+// fp32 scale (|error| <= 2^-12 of the row maximum) and its log2 LSE in fp32.
+// With one split that row is the output.  Otherwise the CTAs that split one
+// row tile's keys form a thread-block cluster: the records are pushed over
+// distributed shared memory into the idle K/V ring of the cluster CTA that
+// owns the row (a split cluster barrier: arrive once the ring is idle, wait
+// before pushing); after a second cluster barrier each CTA merges its slice
+// of rows over the S partials (LSE weights, fixed order) and writes the final
+// bf16 output and LSE.
 //
-// Every wait is bounded (clock64 budget); on expiry the CTA raises
-// TIDAR_DEV_TIMEOUT in dev_status, drains, frees TMEM and returns.
+// Before the previous kernel in the stream has finished (programmatic
+// dependent launch), a CTA sets up its barriers and TMEM and asks L2 for the
+// first K/V tiles of its run, from a prefix length read as a hint; the real
+// copies, and every read the results depend on, wait for that kernel.
+//
+// Every wait is bounded (p.wait_cycles).  On expiry the CTA raises
+// TIDAR_DEV_TIMEOUT in dev_status and every role stops; then the producers
+// wait for their copies in flight and the MMA issuers for their MMAs (bounded
+// waits that ignore the abort), so nothing lands in shared memory or TMEM
+// after the CTA frees it.  No wait sits between two CTA barriers that an
+// aborted warp could skip.
 #include "attn.cuh"
 #include "tc.cuh"
 
@@ -52,11 +63,14 @@ namespace tidar {
 namespace {
 
 constexpr int TM = 128;
-constexpr int TN = 128;
-constexpr int STAGES = 3;
+constexpr int TN = 64;
+constexpr int STAGES = 4;
+constexpr int NSB = 4;  // S buffers: warpgroup w owns buffers w and w + 2
+static_assert(TN == kPageRows, "a KV-cache page is one key tile");
 constexpr int THREADS = 384;
-constexpr int kMaxSplits = 8;  // cluster size limit (portable clusters)
-constexpr long long kWaitCycles = 4000000000LL;
+constexpr int kMaxSplits = 8;                        // cluster size limit (portable clusters)
+constexpr int kPageSlots = kMaxPagesPerSeq + kMaxSplits;  // page ids of one CTA's run of cache tiles
+constexpr long long kDrainCycles = kAttnWaitCycles;  // bound of the waits that drain issued work
 
 template <int D>
 struct Smem {
@@ -65,11 +79,11 @@ struct Smem {
     static constexpr int STAGE = 2 * KV_TILE;
     static constexpr int KV_OFF = Q_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
-    // k_full, k_empty, v_full, v_empty, s_full[3], p_full[3], pv_done[2], o_final, q_full
-    static constexpr int NBARS = 4 * STAGES + 10;
+    // k_full, k_empty, v_full, v_empty, s_full[4], p_full[4], pv_done[4], o_final, q_full, fin_qk, fin_pv, stall
+    static constexpr int NBARS = 4 * STAGES + 3 * NSB + 5;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-    static constexpr int XM_OFF = MISC_OFF + 16;      // row-max exchange between the warpgroups: [2][2][TM] bf16
-    static constexpr int TOTAL = XM_OFF + 2 * 2 * TM * 2;
+    static constexpr int PAGES_OFF = MISC_OFF + 16;  // page ids of the CTA's cache tiles (paged caches)
+    static constexpr int TOTAL = PAGES_OFF + kPageSlots * 4;
     static constexpr int ALLOC = TOTAL + 1024;  // alignment slack
 };
 
@@ -118,8 +132,9 @@ __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv
     for (int kk = 0; kk < TN / 16; ++kk) tc::mma_ts(d_o, a_p + kk * 8, dv + kk * 128, id, (acc || kk > 0) ? 1u : 0u);
 }
 
-// Loads this thread's 64 raw scores (TMEM columns col .. col+63 of its lane) into x.  MASKED: only keys
-// kbase + j in [0, lo) and [glo, ghi) are kept; the others (garbage past the sequence included) become -inf.
+// Loads 64 raw scores (TMEM columns col .. col+63 of this thread's lane, keys kbase .. kbase+63 of the tile)
+// into x.  MASKED: only keys in [0, lo) and [glo, ghi) are kept; the others (garbage past the sequence
+// included) become -inf.
 template <bool MASKED>
 __device__ __forceinline__ void half_load(uint32_t col, int kbase, int lo, int glo, int ghi, float (&x)[64]) {
 #pragma unroll
@@ -141,6 +156,14 @@ __device__ __forceinline__ void half_load(uint32_t col, int kbase, int lo, int g
     }
 }
 
+__device__ __forceinline__ void load_scores(bool masked, uint32_t col, int kbase, int lo, int glo, int ghi,
+                                            float (&x)[64]) {
+    if (masked)
+        half_load<true>(col, kbase, lo, glo, ghi, x);
+    else
+        half_load<false>(col, kbase, lo, glo, ghi, x);
+}
+
 __device__ __forceinline__ float half_max(const float (&x)[64]) {
     float m8[8];  // eight independent chains
 #pragma unroll
@@ -151,28 +174,21 @@ __device__ __forceinline__ float half_max(const float (&x)[64]) {
 }
 
 // p = 2^(x * sl2 + neg_m) for the 64 scores in x (-inf gives exactly 0), written as 32 bf16 pairs to TMEM
-// columns pcol .. pcol+31 (P, the A operand of PV).  Returns the sum of the 64 values of p; *mx receives the
-// maximum of x, computed in the same pass (its ALU work hides under the exponentials).
-__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], float sl2, float neg_m, float *mx) {
-    float sum8[8], m8[8];
+// columns pcol .. pcol+31 (P, the A operand of PV).  Returns the sum of the 64 values of p.
+__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], float sl2, float neg_m) {
+    float sum8[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        sum8[j] = 0.f;
-        m8[j] = -INFINITY;
-    }
+    for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
     uint32_t pk[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const float a = fast_exp2(fmaf(x[2 * j], sl2, neg_m));
         const float bb = fast_exp2(fmaf(x[2 * j + 1], sl2, neg_m));
-        m8[(2 * j) & 7] = fmaxf(m8[(2 * j) & 7], x[2 * j]);
-        m8[(2 * j + 1) & 7] = fmaxf(m8[(2 * j + 1) & 7], x[2 * j + 1]);
         sum8[(2 * j) & 7] += a;
         sum8[(2 * j + 1) & 7] += bb;
         pk[j] = pack_bf16x2(a, bb);
     }
     tc::tmem_st32(pcol, pk);
-    *mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
     return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 }
 
@@ -248,6 +264,14 @@ __device__ __forceinline__ int tile_valid(int t, int TP, int P, int R) {
     return t < TP ? min(TN, P - t * TN) : min(TN, R - (t - TP) * TN);
 }
 
+// Key tiles [t0, t1) of split `split` out of n_splits for a sequence with prefix length P.
+__device__ __forceinline__ void split_range(int P, int R, int split, int n_splits, int &TP, int &t0, int &t1) {
+    TP = ceil_div(P, TN);
+    const int T = TP + ceil_div(R, TN);
+    t0 = (int)((long)split * T / n_splits);
+    t1 = (int)((long)(split + 1) * T / n_splits);
+}
+
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_sm100_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_kc,
@@ -264,19 +288,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto k_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto v_full = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
     auto v_empty = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
-    auto s_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + sb); };      // S buffer sb holds a new S
-    auto p_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + 3 + sb); };  // P in S buffer sb is complete
-    // pv_done(e): its k-th phase completes with PV(2k + e).  Waiting for PV(i) on pv_done(i & 1) is unambiguous
-    // once PV(i-2) has completed, which holds wherever it is waited for (see there).
-    auto pv_done = [&](int e) { return bar0 + 8u * (4 * STAGES + 6 + e); };
-    const uint32_t o_final = bar0 + 8u * (4 * STAGES + 8);  // one phase: the last PV has completed
-    const uint32_t q_full = bar0 + 8u * (4 * STAGES + 9);
+    // Per S buffer sb = i % 4 (tile i is its (i / 4)-th use and completes phase i / 4 of each):
+    auto s_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + sb); };           // S(i) is in buffer sb
+    auto p_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + NSB + sb); };     // P(i) is in buffer sb
+    auto pv_done = [&](int sb) { return bar0 + 8u * (4 * STAGES + 2 * NSB + sb); }; // PV(i) has completed
+    constexpr int X = 4 * STAGES + 3 * NSB;
+    const uint32_t o_final = bar0 + 8u * X;        // one phase: the last PV has completed
+    const uint32_t q_full = bar0 + 8u * (X + 1);
+    const uint32_t fin_qk = bar0 + 8u * (X + 2);   // the QK issuer's MMAs have all completed
+    const uint32_t fin_pv = bar0 + 8u * (X + 3);   // the PV issuer's MMAs have all completed
+    const uint32_t stall = bar0 + 8u * (X + 4);    // nothing arrives here (timeout test)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
     const int split = blockIdx.x, mt = blockIdx.y, bh = blockIdx.z;
     const int b = bh / p.Hkv, kvh = bh % p.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long wl = p.wait_cycles;
     // ---- set-up that needs nothing from the previous kernel (programmatic dependent launch) ----
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -285,20 +313,42 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mbar_init(v_full(s), 1);
             tc::mbar_init(v_empty(s), 1);
         }
-        for (int sb = 0; sb < 3; ++sb) {
+        for (int sb = 0; sb < NSB; ++sb) {
             tc::mbar_init(s_full(sb), 1);
-            tc::mbar_init(p_full(sb), 256);  // both softmax warpgroups
+            tc::mbar_init(p_full(sb), 128);  // the owning warpgroup's threads
+            tc::mbar_init(pv_done(sb), 1);
         }
-        tc::mbar_init(pv_done(0), 1);
-        tc::mbar_init(pv_done(1), 1);
         tc::mbar_init(o_final, 1);
         tc::mbar_init(q_full, q_tma ? 1 : THREADS - 64);
+        tc::mbar_init(fin_qk, 1);
+        tc::mbar_init(fin_pv, 1);
+        tc::mbar_init(stall, 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
         tc::tma_prefetch_desc(&tm_kc);
         tc::tma_prefetch_desc(&tm_vc);
         tc::tma_prefetch_desc(&tm_kn);
         tc::tma_prefetch_desc(&tm_vn);
+        // L2 hint for the first cache tiles of this CTA's run, from the prefix length as it reads now (the
+        // previous kernel may still change it: a wrong guess only costs traffic, L2 stays coherent)
+        const int P_hint = __ldcg(p.prefix_len + b);
+        if (P_hint >= 0 && P_hint <= p.P_max) {
+            int TPh, h0, h1;
+            split_range(P_hint, p.R, split, p.n_splits, TPh, h0, h1);
+            for (int t = h0; t < min(h1, min(h0 + STAGES, TPh)); ++t) {
+                int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
+                if (p.block_table) {
+                    const int pg = __ldcg(p.block_table + (size_t)b * p.max_pages + t);
+                    if (pg < 0 || pg >= p.num_pages) break;
+                    y = (pg * p.Hkv + kvh) * TN;
+                }
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) {
+                    tc::tma_prefetch_l2_2d(&tm_kc, h * 64, y);
+                    tc::tma_prefetch_l2_2d(&tm_vc, h * 64, y);
+                }
+            }
+        }
     }
     if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
     // every global read below (prefix lengths, Q, K/V) waits for the previous kernel
@@ -313,9 +363,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     const int P = p.prefix_len[b];
-    if (P < 0 || P > p.P_max) {
-        if (tid == 0 && split == 0 && mt == 0) atomicOr(p.dev_status, TIDAR_DEV_BAD_PREFIX);
-        if (tid == 0 && q_tma) tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);  // no copy may land after exit
+    int TP, t0, t1;
+    const bool bad_prefix = P < 0 || P > p.P_max;
+    if (!bad_prefix) split_range(P, p.R, split, p.n_splits, TP, t0, t1);
+    int *pages = reinterpret_cast<int *>(smem + L::PAGES_OFF);  // pages[i]: page of cache tile t0 + i
+    bool bad_page = false;
+    if (p.block_table && !bad_prefix) {  // (uniform over the CTA: one sequence)
+        // every CTA of the cluster checks every page of the sequence, so that they all take the same exit (the
+        // early one below passes no cluster barrier); it keeps the ids of its own tiles
+        int bad = 0;
+        for (int t = tid; t < TP; t += THREADS) {
+            const int pg = p.block_table[(size_t)b * p.max_pages + t];
+            bad |= pg < 0 || pg >= p.num_pages;
+            if (t >= t0 && t < t1) pages[t - t0] = pg;
+        }
+        bad_page = __syncthreads_or(bad) != 0;
+    }
+    if (bad_prefix || bad_page) {
+        if (tid == 0 && split == 0 && mt == 0)
+            atomicOr(p.dev_status, bad_prefix ? TIDAR_DEV_BAD_PREFIX : TIDAR_DEV_BAD_PAGE);
+        if (tid == 0 && q_tma) tc::mbar_wait_drain(q_full, 0, kDrainCycles);  // no copy may land after exit
         tc::fence_before_sync();
         __syncthreads();
         if (warp == 1) {
@@ -324,10 +391,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         return;
     }
-    const int TP = ceil_div(P, TN);
-    const int T = TP + ceil_div(p.R, TN);
-    const int t0 = (int)((long)split * T / p.n_splits);
-    const int t1 = (int)((long)(split + 1) * T / p.n_splits);
     const int n = t1 - t0;
 
     // K (is_v = 0) or V (is_v = 1) of tile i into stage i % STAGES of its ring
@@ -338,7 +401,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int t = t0 + i;
         const uint32_t dst = sKV + st * L::STAGE + is_v * L::KV_TILE;
         if (t < TP) {
-            const int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
+            const int y = p.block_table ? (pages[i] * p.Hkv + kvh) * TN : (b * p.Hkv + kvh) * p.P_max + t * TN;
 #pragma unroll
             for (int h = 0; h < D / 64; ++h) tc::tma_load_2d(dst + h * TN * 128, is_v ? &tm_vc : &tm_kc, h * 64, y, bar);
         } else {
@@ -391,24 +454,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                 int issued = prologue;
                 for (int i = prologue; i < n; ++i) {
                     const int u = i / STAGES;
-                    if (!tc::mbar_wait(is_v ? v_empty(i % STAGES) : k_empty(i % STAGES), (u - 1) & 1, abort_flag,
-                                       kWaitCycles))
+                    if (!tc::mbar_wait(is_v ? v_empty(i % STAGES) : k_empty(i % STAGES), (u - 1) & 1, abort_flag, wl))
                         break;
                     issue_tile(i, is_v);
                     issued = i + 1;
                 }
-                // drain: no copy may land after the CTA exits
+                // drain, whatever happened: only the last copy of each stage can still be in flight (an earlier
+                // one completed before its stage was re-armed), and none may land after the CTA exits
                 for (int i = max(0, issued - STAGES); i < issued; ++i)
-                    tc::mbar_wait(is_v ? v_full(i % STAGES) : k_full(i % STAGES), (i / STAGES) & 1, abort_flag,
-                                  kWaitCycles);
+                    tc::mbar_wait_drain(is_v ? v_full(i % STAGES) : k_full(i % STAGES), (i / STAGES) & 1,
+                                        kDrainCycles);
+                if (!is_v && q_tma) tc::mbar_wait_drain(q_full, 0, kDrainCycles);
             }
             __syncwarp();
         } else if (warp == 1 || warp == 3) {
             // ================= MMA issue: QK^T on warp 1, PV on warp 3 (one thread each) =================
-            // Two issuing threads on two SM sub-partitions: each issues half of a tile's MMAs, so neither's
-            // issue rate bounds the tensor pipe.  S of tile j goes to S buffer j % 3.  QK(j), j >= 3, reuses the
-            // buffer whose P PV(j-3) reads, so it is issued once PV(j-3) has completed; with three S buffers that
-            // costs nothing, since the softmax still has S(j-2) and S(j-1) to work on.
             constexpr uint64_t kStage = L::STAGE >> 4;  // one ring stage in the descriptor's address field
             const uint32_t tb = tbase;
             if (lane == 0 && warp == 1) {
@@ -417,19 +477,20 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // low 14 bits (address >> 4; shared memory is < 256 KB, so the add never carries out)
                 const uint64_t dq = tc::smem_desc_sw128(sQ, 16, 1024);
                 const uint64_t dk = tc::smem_desc_sw128(sKV, 16, 1024);
-                bool ok = tc::mbar_wait(q_full, 0, abort_flag, kWaitCycles);
+                bool ok = !p.stall_test || tc::mbar_wait(stall, 0, abort_flag, wl);
+                ok = ok && tc::mbar_wait(q_full, 0, abort_flag, wl);
                 int kst = 0;
                 uint32_t kph = 0;
-                for (int j = 0; j < n && ok; ++j) {
-                    const int sb = j % 3;
-                    if (j >= 3) {  // PV(j-3) done reading P from buffer sb (PV(j-5) was waited for before)
-                        ok = tc::mbar_wait(pv_done((j - 3) & 1), ((j - 3) >> 1) & 1, abort_flag, kWaitCycles);
+                for (int i = 0; i < n && ok; ++i) {
+                    const int sb = i & (NSB - 1);
+                    if (i >= NSB) {  // PV(i-4) has read P out of S buffer sb
+                        ok = tc::mbar_wait(pv_done(sb), ((i >> 2) - 1) & 1, abort_flag, wl);
                         if (!ok) break;
                     }
-                    ok = tc::mbar_wait(k_full(kst), kph, abort_flag, kWaitCycles);
+                    ok = tc::mbar_wait(k_full(kst), kph, abort_flag, wl);
                     if (!ok) break;
                     tc::fence_after_sync();
-                    issue_qk<D>(tb + sb * 128, dq, dk + kst * kStage, id_qk);
+                    issue_qk<D>(tb + sb * TN, dq, dk + kst * kStage, id_qk);
                     tc::mma_commit(s_full(sb));
                     tc::mma_commit(k_empty(kst));
                     if (++kst == STAGES) {
@@ -437,6 +498,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         kph ^= 1u;
                     }
                 }
+                tc::mma_commit(fin_qk);  // every MMA of this thread completes before TMEM is freed
+                tc::mbar_wait_drain(fin_qk, 0, kDrainCycles);
             } else if (lane == 0 && warp == 3) {
                 constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
                 const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
@@ -444,20 +507,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 int vst = 0;
                 uint32_t vph = 0;
                 for (int i = 0; i < n && ok; ++i) {
-                    const int sb = i % 3;
-                    ok = tc::mbar_wait(v_full(vst), vph, abort_flag, kWaitCycles) &&
-                         tc::mbar_wait(p_full(sb), (i / 3) & 1, abort_flag, kWaitCycles);
+                    const int sb = i & (NSB - 1), w = i & 1;
+                    ok = tc::mbar_wait(v_full(vst), vph, abort_flag, wl) &&
+                         tc::mbar_wait(p_full(sb), (i >> 2) & 1, abort_flag, wl);
                     if (!ok) break;
                     tc::fence_after_sync();
-                    issue_pv<D>(tb + 384, tb + sb * 128, dv + vst * kStage, id_pv, i > 0);
+                    issue_pv<D>(tb + 256 + w * 128, tb + sb * TN, dv + vst * kStage, id_pv, i >= 2);
                     tc::mma_commit(v_empty(vst));
-                    tc::mma_commit(pv_done(i & 1));
+                    tc::mma_commit(pv_done(sb));
                     if (i == n - 1) tc::mma_commit(o_final);
                     if (++vst == STAGES) {
                         vst = 0;
                         vph ^= 1u;
                     }
                 }
+                tc::mma_commit(fin_pv);
+                tc::mbar_wait_drain(fin_pv, 0, kDrainCycles);
             }
         }
         __syncwarp();
@@ -472,16 +537,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::tmem_dealloc(tbase, 512);
         }
     } else {
-        // ================= softmax: both warpgroups on every tile =================
-        // Warpgroup w takes columns [64w, 64w+64) of each S tile (thread = query row = TMEM lane).  The two
-        // halves of a row agree on one running max through a small exchange in shared memory, so both scale
-        // their exponentials alike and PV sums them into the one O accumulator.
+        // ================= softmax: warpgroup w on tiles i = w, w+2, ... =================
         const int w = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int m_row = mt * TM + row;
         const int r = m_row / p.G;
-        const int wt = tid - 128;  // 0..255
+        const int wt = tid - 128 - 128 * w;  // 0..127 within the warpgroup
+        // every row of this warp is padding of the last row tile: P = 0, no exponentials
+        const bool pad_warp = mt * TM + q4 * 32 >= p.M;
         // visible new keys of row r: [0, vis_lim) and [vis_glo, vis_ghi) (same rule as new_key_visible)
         int vis_lim, vis_glo = 0, vis_ghi = 0;
         if (p.mask_mode == TIDAR_MASK_CAUSAL || r < p.k) {
@@ -493,16 +557,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             vis_ghi = vis_glo + p.k;
         }
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const uint32_t o_col = tbase + lane_off + 384 + w * (D / 2);  // this warpgroup's half of O
-        __nv_bfloat16 *xm = reinterpret_cast<__nv_bfloat16 *>(smem + L::XM_OFF);  // [2 tiles][2 wg][TM]
+        const uint32_t o_col = tbase + lane_off + 256 + w * 128;  // O_w
         const float sl2 = p.scale_log2;  // > 0, so the max of raw scores gives the max of scaled ones
-        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units, shared by both halves), own sum
+        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units) and sum of this row's tiles
         bool ok = true;
-        for (int i = 0; i < n; ++i) {
-            const int sb = i % 3;
-            if (!tc::mbar_wait(s_full(sb), (i / 3) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
+        for (int i = w; i < n; i += 2) {
+            const int sb = i & (NSB - 1);
+            const uint32_t s_col = tbase + lane_off + sb * TN;  // S buffer of tile i
+            if (ok) ok = tc::mbar_wait(s_full(sb), (i >> 2) & 1, abort_flag, wl);
+            ok = __all_sync(0xffffffffu, ok);  // TMEM accesses are warp-collective: decide per warp
+            if (!ok) continue;                // nothing below waits on other threads: skipping is safe
             tc::fence_after_sync();
-            const uint32_t s_col = tbase + lane_off + sb * 128;
             const int t = t0 + i;
             // a partial prefix tile (keys beyond P) or a new-key tile (the TiDAR mask): the visible keys of
             // this row are [0, lo) and [glo, ghi); everything else, garbage included, is excluded by select
@@ -522,105 +587,104 @@ __global__ void __launch_bounds__(THREADS, 1)
                 lo = min(lo, end);
                 ghi = min(ghi, end);
             }
-            float x[64];
-            if (masked)
-                half_load<true>(s_col + w * 64, w * 64, lo, glo, ghi, x);
-            else
-                half_load<false>(s_col + w * 64, w * 64, lo, glo, ghi, x);
-            // Exponentials against the running max the two halves already share (stale by design: exact as long
-            // as p <= 2^8); the tile's row max comes out of the same pass.  Only a row whose max grew by more
-            // than 2^8 -- all rows on the first tile, rarely later -- redoes them with the new max.
-            const uint32_t pcol = s_col + w * 32;  // P of keys [64w, 64w+64) over S columns [32w, 32w+32)
-            const bool fresh = m_run == -INFINITY;  // no visible key so far: no max to reuse
-            float hmx;
-            float lt = fresh ? 0.f : half_exp(pcol, x, sl2, -m_run, &hmx);
-            if (fresh) hmx = half_max(x);
-            // both halves' maxima (rounded to bf16 for the exchange: any value the two sides agree on and that
-            // is within 2^8 of the true maximum serves)
-            const __nv_bfloat16 hb = __float2bfloat16_rn(hmx);
-            xm[((i & 1) * 2 + w) * TM + row] = hb;
-            asm volatile("bar.sync 1, 256;\n" ::: "memory");
-            const __nv_bfloat16 ob = xm[((i & 1) * 2 + (1 - w)) * TM + row];
-            const float mx = fmaxf(__bfloat162float(hb), __bfloat162float(ob)) * sl2;
-            const float m_new = fmaxf(m_run, mx);
-            const bool grow = m_new > m_run + 8.f;
-            if (__any_sync(0xffffffffu, grow || fresh)) {  // fresh rows have written no P yet
-                if (i >= 1 && __any_sync(0xffffffffu, grow)) {
-                    // rescale this half of O once PV(i-1), the last to write it, has completed.  S(i) is
-                    // complete, and QK(i) was issued after PV(i-3) completed: the wait below is unambiguous.
-                    if (!tc::mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, kWaitCycles)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
-                    const float f = grow ? fast_exp2(m_run - m_new) : 1.f;
-#pragma unroll 1
-                    for (int c = 0; c < D / 64; ++c) {
-                        uint32_t v[32];
-                        tc::tmem_ld32(o_col + c * 32, v);
-                        tc::tmem_wait_ld();
+            if (pad_warp) {
+                uint32_t z[32];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-                        tc::tmem_st32(o_col + c * 32, v);
+                for (int j = 0; j < 32; ++j) z[j] = 0u;
+                tc::tmem_st32(s_col, z);
+            } else {
+                float x[64];
+                load_scores(masked, s_col, 0, lo, glo, ghi, x);
+                const float mx = half_max(x) * sl2;  // the tile's row max
+                // the running max moves only when the tile's max exceeds it by more than 2^8 (always on the
+                // first tile with a visible key)
+                const bool grow = mx > m_run + 8.f;
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float m_new = grow ? mx : m_run;
+                    const float f = grow ? fast_exp2(m_run - m_new) : 1.f;  // 0 when m_run = -inf
+                    if (i >= 2) {
+                        // rescale O_w, last written by PV(i-2) (complete: QK(i) was issued after PV(i-4), and
+                        // the wait below makes the order explicit)
+                        const int ip = i - 2;
+                        bool ok2 = tc::mbar_wait(pv_done(ip & (NSB - 1)), (ip >> 2) & 1, abort_flag, wl);
+                        ok = __all_sync(0xffffffffu, ok2);
+                        if (!ok) continue;
+                        tc::fence_after_sync();
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t v[32];
+                            tc::tmem_ld32(o_col + c * 32, v);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+                            tc::tmem_st32(o_col + c * 32, v);
+                        }
                     }
-                }
-                if (grow) {
-                    l_run *= fast_exp2(m_run - m_new);
+                    l_run *= f;
                     m_run = m_new;
                 }
-                tc::tmem_wait_st();  // the redone P overwrites the first pass's
-                float unused;
-                lt = half_exp(pcol, x, sl2, m_run == -INFINITY ? 0.f : -m_run, &unused);
+                // exponentials: P of the tile's 64 keys goes to the first 32 columns of its S buffer
+                l_run += half_exp(s_col, x, sl2, m_run == -INFINITY ? 0.f : -m_run);
             }
-            l_run += lt;
             const int valid = tile_valid(t, TP, P, p.R);
             if (valid < TN) {
                 // keys past the sequence: zero their V rows (0 * garbage could be NaN) before PV reads them
                 const int st = i % STAGES;
-                if (!tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, kWaitCycles)) { ok = false; break; }
-                uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
-                for (int idx = wt; idx < (TN - valid) * (D / 8); idx += 256) {
-                    const int j = valid + idx / (D / 8), c = idx % (D / 8);
-                    *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
-                        make_uint4(0, 0, 0, 0);
+                bool ok2 = tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, wl);
+                ok = __all_sync(0xffffffffu, ok2);
+                if (ok) {
+                    uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
+                    for (int idx = wt; idx < (TN - valid) * (D / 8); idx += 128) {
+                        const int j = valid + idx / (D / 8), c = idx % (D / 8);
+                        *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    tc::fence_proxy_async_smem();
                 }
-                tc::fence_proxy_async_smem();
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            tc::mbar_arrive(p_full(sb));
+            if (ok) tc::mbar_arrive(p_full(sb));
         }
+        tc::tmem_wait_st();  // (abort path) no TMEM store left in flight
         // the next kernel in the stream may launch now: it waits for this grid before touching memory
         asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
         constexpr int H = D / 2;
-        if (ok && n > 0) ok = tc::mbar_wait(o_final, 0, abort_flag, kWaitCycles);  // O final
+        bool fin = ok && n > 0 && tc::mbar_wait(o_final, 0, abort_flag, wl);  // O final
+        fin = __all_sync(0xffffffffu, fin);
         tc::fence_after_sync();
         // this CTA's K/V ring is idle: once every CTA of the cluster has arrived here, the others may write
         // their partial records into it (the wait is just before the push below).  The arrival publishes
         // nothing, so it carries no release fence.
         tc::cluster_arrive_relaxed();
-        // the row sum is split over the two halves
-        float *xl = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM]
-        xl[w * TM + row] = l_run;
+        // the two accumulators of a row: O = (2^(m_0 - m) O_0 + 2^(m_1 - m) O_1) / l, l = the weighted sums
+        float *xs = reinterpret_cast<float *>(smem + L::KV_OFF);  // [4][TM]: m_0, l_0, m_1, l_1
+        xs[(2 * w) * TM + row] = m_run;
+        xs[(2 * w + 1) * TM + row] = l_run;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        const float lt = l_run + xl[(1 - w) * TM + row];
+        const float m0 = xs[row], l0 = xs[TM + row], m1 = xs[2 * TM + row], l1 = xs[3 * TM + row];
+        const float mm = fmaxf(m0, m1);
+        const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
+        const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
+        const float lt = a0 * l0 + a1 * l1;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float lse2 = lt > 0.f ? m_run + __log2f(lt) : -INFINITY;  // log2 of this CTA's row sum
-        // tcgen05.ld is warp-collective: the decision to read the accumulator must be warp-uniform
-        const bool rd = __all_sync(0xffffffffu, ok && n > 0);
-        uint32_t va[H / 32][32];
-#pragma unroll
-        for (int c = 0; c < H / 32; ++c) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) va[c][j] = 0u;
-            if (rd) tc::tmem_ld32(o_col + c * 32, va[c]);
-        }
-        tc::tmem_wait_ld();
+        const float lse2 = lt > 0.f ? mm + __log2f(lt) : -INFINITY;  // log2 of this CTA's row sum
+        const bool has1 = n >= 2;  // O_1 was written only if warpgroup 1 had a tile
+        const float f0 = a0 * inv, f1 = has1 ? a1 * inv : 0.f;
         float hv[H];
 #pragma unroll
-        for (int c = 0; c < H / 32; ++c)
+        for (int c = 0; c < H / 32; ++c) {
+            uint32_t v0[32], v1[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) hv[c * 32 + j] = rd ? __uint_as_float(va[c][j]) * inv : 0.f;
+            for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0u;
+            const uint32_t col = tbase + lane_off + 256 + w * H + c * 32;  // this warpgroup's half of the columns
+            if (fin) tc::tmem_ld32(col, v0);
+            if (fin && has1) tc::tmem_ld32(col + 128, v1);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                hv[c * 32 + j] = fin ? f0 * __uint_as_float(v0[j]) + (has1 ? f1 * __uint_as_float(v1[j]) : 0.f) : 0.f;
+        }
         const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
         // CTA s of the cluster merges rows [s*per, (s+1)*per) of the tile; it receives every CTA's partial
         // record of those rows in its (idle) ring: vals [S][D/8][per] 16-byte chunks (8 fp16 of one row),
@@ -712,7 +776,9 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims
 template <int D>
 cudaError_t launch(const AttnParams &p, cudaStream_t s) {
     CUtensorMap kc, vc, kn, vn, qm;
-    const cuuint64_t dc[2] = {(cuuint64_t)D, (cuuint64_t)p.B * p.Hkv * p.P_max};
+    const cuuint64_t cache_rows =
+        p.block_table ? (cuuint64_t)p.num_pages * p.Hkv * TN : (cuuint64_t)p.B * p.Hkv * p.P_max;
+    const cuuint64_t dc[2] = {(cuuint64_t)D, cache_rows};
     const cuuint64_t sc[1] = {(cuuint64_t)D * 2};
     const cuuint32_t bc[2] = {64, TN};
     const cuuint64_t dn[3] = {(cuuint64_t)D, (cuuint64_t)p.Hkv, (cuuint64_t)p.B * p.R};

@@ -16,6 +16,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kNumSMs = 148;
 constexpr int kMaxDraft = 16;  // longest draft block k every entry point accepts
+constexpr int kPageRows = 64;  // rows of a KV-cache page: one key tile of the attention kernel
+constexpr int kMaxPagesPerSeq = 1024;  // longest block-table row a paged call accepts (65536 cached tokens)
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

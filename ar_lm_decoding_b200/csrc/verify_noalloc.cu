@@ -13,8 +13,10 @@
 // current, resolves the real address with cudaGetSymbolAddress and caches it;
 // that first call should therefore come before any stream capture.  Every
 // call on a device shares the same array: calls whose kernels overlap on the
-// GPU (other streams, or no ordering between them) race on it.  Nothing in the
-// array needs to start at zero -- each call writes every entry it later reads.
+// GPU (other streams, or no ordering between them) race on it.  The one entry
+// that must start at zero, the verify kernel's grid-barrier counter, is
+// cleared in stream order at the start of every call (cudaMemsetAsync, which
+// allocates nothing); every other entry is written before it is read.
 #include <mutex>
 
 #include "common.cuh"
@@ -22,8 +24,8 @@
 namespace tidar {
 size_t verify_workspace_bytes(int B, int k, int V);
 cudaError_t verify_launch(const void *, const void *, int, const int32_t *, const uint8_t *, const float *,
-                          const float *, int, int, int, int32_t *, int32_t *, int32_t *, int32_t *, float *, float *,
-                          void *, int32_t *, cudaStream_t);
+                          const float *, int, int, int, float, int32_t *, int32_t *, int32_t *, int32_t *, float *,
+                          float *, void *, int32_t *, cudaStream_t);
 }  // namespace tidar
 
 namespace {
@@ -73,8 +75,8 @@ tidar_status tidar_verify_noalloc(const void *p_logits, const void *q_logits, in
     void *scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return TIDAR_ERR_CUDA;
     const cudaError_t e = tidar::verify_launch(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u_res, B,
-                                               k, V, accept_len, resampled, tokens, n_emitted, logp_d, logq_d, scratch,
-                                               dev_status, static_cast<cudaStream_t>(stream));
+                                               k, V, 1.f, accept_len, resampled, tokens, n_emitted, logp_d, logq_d,
+                                               scratch, dev_status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TIDAR_OK : TIDAR_ERR_CUDA;
 }
 

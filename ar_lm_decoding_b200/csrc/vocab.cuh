@@ -90,10 +90,9 @@ __device__ __forceinline__ double block_sum_d(double v, double *red) {
     return r;
 }
 
-// Statistics (max, sum exp) of chunk c of one logit row; every thread returns them.
-__device__ __forceinline__ ChunkStat chunk_stat(const void *row, int dtype, int V, int c, float *redf, double *redd) {
-    float v[32];
-    load_chunk32(row, dtype, V, c, v);
+// Statistics (max, sum exp) of the 32 values of every thread of the block (missing entries -inf); every
+// thread returns them.
+__device__ __forceinline__ ChunkStat stat_of(const float (&v)[32], float *redf, double *redd) {
     float mx = -INFINITY;
 #pragma unroll
     for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
@@ -107,6 +106,52 @@ __device__ __forceinline__ ChunkStat chunk_stat(const void *row, int dtype, int 
     st.pad = 0.f;
     st.z = block_sum_d<kStatThreads>((double)s, redd);
     return st;
+}
+
+// Statistics (max, sum exp) of chunk c of one logit row; every thread returns them.
+__device__ __forceinline__ ChunkStat chunk_stat(const void *row, int dtype, int V, int c, float *redf, double *redd) {
+    float v[32];
+    load_chunk32(row, dtype, V, c, v);
+    return stat_of(v, redf, redd);
+}
+
+// The verify's target logits from an AR value zp and a diffusion value zq: lambda * zp + (1 - lambda) * zq,
+// with the endpoints taken as stored (an infinite logit never meets a zero weight).
+__device__ __forceinline__ float mix_logit(float zp, float zq, float lambda) {
+    if (lambda == 1.f) return zp;
+    if (lambda == 0.f) return zq;
+    return fmaf(lambda, zp, (1.f - lambda) * zq);
+}
+
+// Grid-wide barrier of a cooperative launch: every CTA arrives on `counter` (zeroed before the launch, one
+// increment per CTA per barrier) and waits until it reaches `target`.  The wait is bounded: after `limit`
+// clock cycles the CTA raises TIDAR_DEV_TIMEOUT and returns false.  Writes before the barrier are visible to
+// reads after it in every CTA (release on arrival, acquire on the wait; read such data with __ldcg).
+__device__ __forceinline__ bool grid_barrier(unsigned *counter, unsigned target, int32_t *dev_status,
+                                             long long limit) {
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;\n" ::"l"(counter) : "memory");
+        int ok = 1;
+        const long long t0 = clock64();
+        while (true) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(counter) : "memory");
+            if (v >= target) break;
+            if (clock64() - t0 > limit) {
+                atomicOr(dev_status, TIDAR_DEV_TIMEOUT);
+                ok = 0;
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
 }
 
 // This thread's 32 consecutive entries (tid*32 .. tid*32+31) of chunk c (256 threads), -inf beyond V.
@@ -184,11 +229,13 @@ __device__ __forceinline__ int chunk_search256(const double (&w)[32], double tar
 __device__ __forceinline__ void merge_stats_warp(const ChunkStat *st, int n, float &m, double &z) {
     const int lane = threadIdx.x & 31;
     float mx = -INFINITY;
-    for (int c = lane; c < n; c += 32) mx = fmaxf(mx, st[c].m);
+    for (int c = lane; c < n; c += 32) mx = fmaxf(mx, __ldcg(&st[c].m));
     m = warp_max(mx);
     double s = 0.0;
-    for (int c = lane; c < n; c += 32)
-        if (st[c].m != -INFINITY) s += st[c].z * (double)exp2f((st[c].m - m) * kLog2e);
+    for (int c = lane; c < n; c += 32) {
+        const float mc = __ldcg(&st[c].m);
+        if (mc != -INFINITY) s += __ldcg(&st[c].z) * (double)exp2f((mc - m) * kLog2e);
+    }
     z = warp_sum_d(s);
 }
 

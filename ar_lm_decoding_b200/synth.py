@@ -81,6 +81,10 @@ CONFIGS = {
     "qwen3-32b_k4": StepConfig("qwen3-32b_k4", L=64, Hq=64, Hkv=8, D=128, P=16384, k=4, V=151936, cfg_id=5),
     "qwen3-32b_k8": StepConfig("qwen3-32b_k8", L=64, Hq=64, Hkv=8, D=128, P=16384, k=8, V=151936, cfg_id=6),
     "qwen3-32b_k16": StepConfig("qwen3-32b_k16", L=64, Hq=64, Hkv=8, D=128, P=16384, k=16, V=151936, cfg_id=7),
+    # the Qwen3-8B step once more with the planted-peak logits of the Qwen2.5 workloads, so that accept lengths
+    # vary and the commit copies rows
+    "qwen3-8b_k8_peaks": StepConfig("qwen3-8b_k8_peaks", L=36, Hq=32, Hkv=8, D=128, P=4096, k=8, V=151936, peaks=True,
+                                    cfg_id=8),
 }
 
 

@@ -320,9 +320,9 @@ def job_throughput(world, step_s):
 
 
 def kernels_per_step(cfg):
-    # per layer: one attention kernel (split-KV merged in-kernel); verify: 2 (vocab statistics, decision);
-    # commit: 1 (its counters are zeroed by a memset node, not a kernel)
-    return cfg.L + 2 + 1
+    # per layer: one attention kernel (split-KV merged in-kernel); verify: one cooperative kernel; commit: one
+    # cooperative kernel (their grid-barrier counters are zeroed by memset nodes, not kernels)
+    return cfg.L + 2
 
 
 def init_ranks(backend):
@@ -434,6 +434,10 @@ def gpu_arm(args, cfg):
     torch.cuda.synchronize()
     attn_ms_launch = max_over_ranks(a0.elapsed_time(a1) / (reps * cfg.L))
     del attn_graph
+    breakdown = {"attn_us_per_launch": round(attn_ms_launch * 1e3, 3),
+                 "verify_us": round(graph_us(stream, reps, lambda: step.verify(stream.cuda_stream)), 3),
+                 "commit_us": round(graph_us(stream, reps, lambda: (step.prefix.copy_(step.prefix0),
+                                                                    step.commit(stream.cuda_stream))), 3)}
 
     e2e = e2e_leg(step, stream, args, barrier, max_over_ranks, world)
 
@@ -483,6 +487,7 @@ def gpu_arm(args, cfg):
                                           4),
                      "peak_kind": peak_kind},
         "clocks": ck,
+        "breakdown": breakdown,
         "e2e": e2e,
         "gpu_launches": kernels_per_step(cfg) * args.steps,
         "accept_len": accept.tolist(),
@@ -493,6 +498,26 @@ def gpu_arm(args, cfg):
     if world > 1:
         dist.destroy_process_group()
     return res if rank == 0 else None
+
+
+def graph_us(stream, reps, fn):
+    """Average duration of `fn`'s launches captured alone in a CUDA graph on `stream` (events on that stream)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / reps
 
 
 def e2e_step(step, stream, copy_stream, events, pin_in, pin_out):
@@ -552,7 +577,7 @@ def check_line(res):
     cannot exceed the device-timed rate; the dominant kernel cannot take longer than the step."""
     assert res["e2e"]["value"] <= res["value"] * 1.02, (res["e2e"]["value"], res["value"])
     us_attn = res["roofline"]["us_per_launch"]
-    assert us_attn * (res["gpu_launches"] / res["steps"] - 3) <= res["ms_per_step"] * 1e3 * 1.05, res
+    assert us_attn * (res["gpu_launches"] / res["steps"] - 2) <= res["ms_per_step"] * 1e3 * 1.05, res
 
 
 def load_traffic(cfg):
@@ -759,6 +784,125 @@ def free_port():
         return s.getsockname()[1]
 
 
+def k_sweep(args, cfg):
+    """Step latency against the draft length k at the workload's other sizes (one JSON line per k): where the
+    step leaves the memory-bound regime (the TiDAR summary's Fig. 1 observation of free token slots, here for
+    this B200 step), and the draft length the step-latency model picks for a few per-draft acceptance rates
+    (tidar_pick_draft_length)."""
+    import torch
+    from ar_lm_decoding_b200 import abi
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    peaks, _ = load_peaks()
+    hbm, tf = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    ks = [int(x) for x in args.ks.split(",")]
+    table = [0.0] * max(ks)
+    for k in ks:
+        c = cfg.with_(k=k)
+        step = Step(c, device)
+        stream = torch.cuda.Stream(device)
+        with torch.cuda.stream(stream):
+            step.run(stream.cuda_stream)
+        torch.cuda.synchronize()
+        assert step.status.item() == 0
+        reps = max(3, min(args.steps, 50))
+        us = graph_us(stream, reps, lambda: step.run(stream.cuda_stream))
+        attn = graph_us(stream, reps, lambda: [step.attn(l, stream.cuda_stream) for l in range(c.L)]) / c.L
+        byts = algorithmic_bytes(c, step.prefix_sum)
+        flops = attn_flops(c, step.prefix_sum)
+        table[k - 1] = us
+        print(json.dumps({"mode": "k_sweep", "workload": workload_desc(c, c.B), "k": k, "query_rows": c.R,
+                          "tokens_per_forward": c.R, "step_us": round(us, 2), "attn_us_per_launch": round(attn, 3),
+                          "hbm_bound_us": round((byts["kv"] + byts["qkvo"] + byts["logits"]) / hbm / 1e3, 2),
+                          "tensor_bound_us": round(flops / tf / 1e6, 2),
+                          "kv_logit_frac": round((byts["kv"] + byts["logits"]) / (us * 1e-6) / 1e9 / hbm, 4),
+                          "tensor_frac": round(flops / (us * 1e-6) / 1e12 / tf, 4)}), flush=True)
+        del step
+        torch.cuda.empty_cache()
+    picks = {}
+    for alpha in (0.3, 0.5, 0.7, 0.8, 0.9, 0.95):
+        k, rate = abi.tidar_pick_draft_length(table, alpha)
+        picks[str(alpha)] = {"k": k, "tokens_per_ms": round(rate * 1e3, 3)}
+    print(json.dumps({"mode": "k_sweep_pick", "workload": cfg.name, "measured_k": ks, "pick": picks}), flush=True)
+
+
+QWEN3_32B_LAYER = {"hidden": 5120, "intermediate": 25600, "Hq": 64, "Hkv": 8, "D": 128}
+
+
+def layer_sweep(args, cfg):
+    """Latency of one full decoder layer against the tokens per forward R = k(k+2), at several prefix lengths:
+    the QKV projection (cuBLAS GEMM), the rotary embedding fused with the re-layout into the attention inputs
+    (tidar_rope_qkv), the hybrid-mask attention (tidar_attn_step), the output projection and the MLP GEMMs
+    (cuBLAS), with synthetic bf16 weights of the Qwen3-32B shape.  This is the B200 counterpart of the TiDAR
+    summary's Fig. 1 (latency against tokens per forward: flat while the weights and the KV cache dominate,
+    rising once the layer is compute-bound); the norms and the activation are left out (elementwise work that
+    does not move the curve).  One JSON line per (prefix, k)."""
+    import torch
+    from ar_lm_decoding_b200 import abi
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    sh = QWEN3_32B_LAYER
+    hid, inter, Hq, Hkv, D = sh["hidden"], sh["intermediate"], sh["Hq"], sh["Hkv"], sh["D"]
+    g = torch.Generator(device=device).manual_seed(0)
+
+    def w(n_in, n_out):
+        return (torch.randn(n_in, n_out, generator=g, device=device) * n_in ** -0.5).to(torch.bfloat16)
+
+    w_qkv, w_o = w(hid, (Hq + 2 * Hkv) * D), w(Hq * D, hid)
+    w_gu, w_down = w(hid, 2 * inter), w(inter, hid)
+    weight_bytes = 2 * sum(t.numel() for t in (w_qkv, w_o, w_gu, w_down))
+    peaks, _ = load_peaks()
+    hbm, tf = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    stream = torch.cuda.Stream(device)
+    ks = [int(x) for x in args.ks.split(",")]
+    for P in [int(x) for x in args.prefixes.split(",")]:
+        P_max = (P + 16 + 63) // 64 * 64
+        kc = torch.randn(1, Hkv, P_max, D, generator=g, device=device).to(torch.bfloat16)
+        vc = torch.randn(1, Hkv, P_max, D, generator=g, device=device).to(torch.bfloat16)
+        pl = torch.tensor([P], dtype=torch.int32, device=device)
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        for k in ks:
+            R = k * (k + 2)
+            x = torch.randn(R, hid, generator=g, device=device).to(torch.bfloat16)
+            qkv = torch.empty(R, (Hq + 2 * Hkv) * D, dtype=torch.bfloat16, device=device)
+            q = torch.empty(1, R, Hq, D, dtype=torch.bfloat16, device=device)
+            kn = torch.empty(1, R, Hkv, D, dtype=torch.bfloat16, device=device)
+            vn = torch.empty(1, R, Hkv, D, dtype=torch.bfloat16, device=device)
+            o = torch.empty(1, R, Hq, D, dtype=torch.bfloat16, device=device)
+            lse = torch.empty(1, R, Hq, dtype=torch.float32, device=device)
+
+            def layer(with_attn=True):
+                torch.matmul(x, w_qkv, out=qkv)
+                abi.tidar_rope_qkv(qkv, pl, 1, Hq, Hkv, D, k, 1e6, q, kn, vn, st, stream.cuda_stream)
+                if with_attn:
+                    abi.tidar_attn_step(q, kn, vn, kc, vc, pl, 1, Hq, Hkv, D, k, P_max, D ** -0.5,
+                                        abi.TIDAR_MASK_HYBRID, o, lse, None, 0, st, stream.cuda_stream)
+                h = torch.matmul(o.view(R, Hq * D), w_o)
+                gu = torch.matmul(h, w_gu)
+                torch.matmul(gu[:, :inter], w_down)
+
+            with torch.cuda.stream(stream):
+                layer()
+            torch.cuda.synchronize()
+            assert st.item() == 0
+            reps = max(3, min(args.steps, 30))
+            us = graph_us(stream, reps, layer)
+            attn_us = graph_us(stream, reps, lambda: abi.tidar_attn_step(
+                q, kn, vn, kc, vc, pl, 1, Hq, Hkv, D, k, P_max, D ** -0.5, abi.TIDAR_MASK_HYBRID, o, lse, None, 0, st,
+                stream.cuda_stream))
+            rope_us = graph_us(stream, reps, lambda: abi.tidar_rope_qkv(qkv, pl, 1, Hq, Hkv, D, k, 1e6, q, kn, vn, st,
+                                                                        stream.cuda_stream))
+            flops = 2 * R * weight_bytes / 2 + 4 * Hq * R * D * P
+            byts = weight_bytes + 4 * Hkv * D * P
+            print(json.dumps({"mode": "layer_sweep", "shape": "Qwen3-32B layer (hidden 5120, intermediate 25600, "
+                              "Hq 64 / Hkv 8, D 128), batch 1", "prefix": P, "k": k, "tokens_per_forward": R,
+                              "layer_us": round(us, 2), "attn_us": round(attn_us, 2), "rope_us": round(rope_us, 2),
+                              "hbm_bound_us": round(byts / hbm / 1e3, 2),
+                              "tensor_bound_us": round(flops / tf / 1e6, 2)}), flush=True)
+        del kc, vc
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser()
@@ -771,6 +915,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--attn-prefix-sweep", action="store_true",
                     help="print attention time per launch against the prefix length (not the benchmark line)")
+    ap.add_argument("--k-sweep", action="store_true",
+                    help="print the step latency for each draft length in --ks (not the benchmark line)")
+    ap.add_argument("--ks", default="1,2,4,8,12,16")
+    ap.add_argument("--layer-sweep", action="store_true",
+                    help="print one full decoder layer's latency against tokens per forward (not the benchmark line)")
+    ap.add_argument("--prefixes", default="1024,4096,16384")
     ap.add_argument("--replica-dry-run", action="store_true",
                     help="run only the replica bookkeeping on CPU (gloo) and print its fields (no GPU work)")
     args = ap.parse_args(argv)
@@ -790,6 +940,12 @@ def main(argv=None):
         return 0
     if args.attn_prefix_sweep:
         attn_prefix_sweep(args, cfg)
+        return 0
+    if args.k_sweep:
+        k_sweep(args, cfg)
+        return 0
+    if args.layer_sweep:
+        layer_sweep(args, cfg)
         return 0
     if world is None and args.gpus > 1:
         # not under a launcher: start the N replicas (one process per GPU) and pass on their exit status

@@ -57,6 +57,7 @@ typedef enum {
 #define TIDAR_DEV_BAD_TOKEN 2  /* a draft or resampled token outside [0, V) */
 #define TIDAR_DEV_BAD_ACCEPT 4 /* accept_len[b] outside [0, k] */
 #define TIDAR_DEV_TIMEOUT 8    /* a bounded on-chip wait expired; the outputs are not valid */
+#define TIDAR_DEV_BAD_PAGE 16  /* a block-table entry outside [0, num_pages) (paged caches) */
 
 typedef enum { TIDAR_DT_BF16 = 0, TIDAR_DT_F32 = 1 } tidar_dtype;
 
@@ -111,6 +112,53 @@ tidar_status tidar_attn_step(const void *q, const void *k_new, const void *v_new
                              int mask_mode, void *out, float *lse, void *workspace, size_t ws_bytes,
                              int32_t *dev_status, void *stream);
 
+/*
+ * tidar_attn_step over a paged KV cache.
+ *
+ * Defined by: as tidar_attn_step; the paging is the serving layout the TiDAR
+ * summary names as the next step beyond its batch-1 runs ("局限与 Future Work":
+ * batch > 1, continuous batching and PagedAttention left untested).  Cache row
+ * n of sequence b is row n % 64 of page block_table[b * max_pages + n / 64] of
+ * the pools:
+ *
+ * k_pool, v_pool  bf16 [num_pages, Hkv, 64, D]: pages shared by all sequences;
+ *                 a sequence's pages need not be contiguous or ordered
+ * block_table     int32 [B, max_pages] (device): page ids of each sequence's
+ *                 cache rows, in row order; entries past ceil(P_b / 64) are
+ *                 not read.  1 <= max_pages <= 1024 (P_b <= 64 * max_pages).
+ * Everything else as tidar_attn_step (no workspace).  A page id outside
+ * [0, num_pages) sets TIDAR_DEV_BAD_PAGE and that sequence is skipped.  The
+ * results equal tidar_attn_step's on the same rows laid out contiguously.
+ */
+tidar_status tidar_attn_step_paged(const void *q, const void *k_new, const void *v_new,
+                                   const void *k_pool, const void *v_pool, const int32_t *block_table,
+                                   int max_pages, int num_pages, const int32_t *prefix_len,
+                                   int B, int Hq, int Hkv, int D, int k, float softmax_scale,
+                                   int mask_mode, void *out, float *lse, int32_t *dev_status, void *stream);
+
+/*
+ * Rotary position embedding of one step's rows, fused with the re-layout of the
+ * QKV projection output into tidar_attn_step's inputs (q, k_new, v_new).
+ *
+ * Defined by: the Qwen backbones the TiDAR pages start from (summary, 核心方法 /
+ * initialisation: Qwen2.5-1.5B, Qwen3-8B; rotary embedding, base theta = 1e6
+ * for both) and the step layout of summary §3.2.  Row positions (the pages
+ * give the partitions, not the positions): draft d_i at P_b + i - 1; slot s of
+ * pre-draft group j at P_b + j + s.  Pair (x_i, x_{i+D/2}), i < D/2, of every
+ * query and key head is rotated by pos * theta^(-2i/D); value heads are copied.
+ * The rotation is computed in double precision and rounded once to bf16.
+ *
+ * qkv        bf16 [B, R, Hq + 2 Hkv, D]: Q heads, then K heads, then V heads
+ * prefix_len int32 [B] (device)
+ * theta      rotary base, > 1
+ * q          bf16 [B, R, Hq, D]; k_new, v_new bf16 [B, R, Hkv, D]
+ * D in {64, 128}, Hq % Hkv == 0, k in 1..16; all tensors 16-byte aligned.
+ * dev_status TIDAR_DEV_BAD_PREFIX (and that sequence's Q/K left unwritten) for
+ *            a negative prefix length.
+ */
+tidar_status tidar_rope_qkv(const void *qkv, const int32_t *prefix_len, int B, int Hq, int Hkv, int D, int k,
+                            double theta, void *q, void *k_new, void *v_new, int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Verify                                                                    */
 /* ------------------------------------------------------------------------ */
@@ -150,6 +198,32 @@ tidar_status tidar_verify(const void *p_logits, const void *q_logits, int logits
                           int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
                           float *logp_d, float *logq_d, void *workspace, size_t ws_bytes,
                           int32_t *dev_status, void *stream);
+
+/*
+ * tidar_verify with a trust-mixed target.
+ *
+ * Defined by: TiDAR summary, "Trust AR vs trust diffusion logits (验证时混合)"
+ * (Fig. 6: the AR and diffusion logits are mixed with a weight lambda at
+ * verification; quality barely moves across lambda) and the notes.yuuk.io talk
+ * notes §生成評価 ("Trust Diff" mode).  The target of the rejection test of slot
+ * i becomes p_i = softmax(trust_ar * p_logits_i + (1 - trust_ar) * q_logits_i)
+ * (q_logits_i, the stored diffusion logits that proposed d_i, serve as the
+ * diffusion logits of that position): draft d_i is accepted with probability
+ * min(1, p_i(d_i)/q_i(d_i)) and a rejection draws from norm(max(0, p_i - q_i)).
+ * trust_ar = 1 is tidar_verify; trust_ar = 0 accepts every draft.  The mix is
+ * formed in fp32 from the stored logits; at the endpoints the stored row is
+ * used as is.
+ *
+ * trust_ar   in [0, 1], else TIDAR_ERR_INVALID_ARG.  logp_d receives
+ *            log p_i(d_i) of the mixed target.  Everything else as tidar_verify
+ *            (same workspace size).
+ */
+tidar_status tidar_verify_trust_mix(const void *p_logits, const void *q_logits, int logits_dtype,
+                                    const int32_t *drafts, const uint8_t *preaccepted,
+                                    const float *u_acc, const float *u_res, int B, int k, int V, float trust_ar,
+                                    int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
+                                    float *logp_d, float *logq_d, void *workspace, size_t ws_bytes,
+                                    int32_t *dev_status, void *stream);
 
 /*
  * tidar_verify without a caller workspace.  The paper has no counterpart: this
@@ -217,6 +291,58 @@ tidar_status tidar_kv_commit(void *const *k_caches, void *const *v_caches,
                              const void *group_logits, int logits_dtype, int V, const float *u_draft,
                              int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group,
                              void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Draft length (host functions, no device work)                             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Expected number of tokens one decode step emits in steady state when every
+ * draft is accepted independently with probability alpha, at draft length k.
+ *
+ * Defined by: the decode step of this library (summary §3.2: a rejected draft
+ * is replaced by a draw from the residual; the pre-drafts of group j* become
+ * the next drafts), read as a two-state chain: a step with a pre-accepted slot
+ * 1 (the previous step's resampled token, already emitted) tests k - 1 drafts,
+ * one without tests k.  Testing m drafts emits sum_{i=1..m} alpha^i + (1 -
+ * alpha^m) new tokens on average (the accepted drafts, then the resampled
+ * token unless all m were accepted).  Returns E, or -1 for k outside 1..16 or
+ * alpha outside [0, 1].
+ */
+double tidar_expected_tokens_per_step(int k, double alpha);
+
+/*
+ * Draft length that maximises expected tokens per microsecond.
+ *
+ * Defined by: the summary's "局限与 Future Work" (Future work 2: choose the
+ * draft block to fit the GPU's free token slots) and the zero-shot draft
+ * length of §3.3 (the draft length can change at inference time).
+ * step_us[k-1] (host array of n <= 16 doubles) is the latency of one decode
+ * step at draft length k -- measured (bench.py --k-sweep) or from a roofline
+ * model; entries <= 0 or non-finite are skipped.  Returns the k in 1..n with
+ * the largest tidar_expected_tokens_per_step(k, alpha) / step_us[k-1] (the
+ * shorter k on a tie) and writes that rate to *tokens_per_us (nullable); 0 on
+ * invalid arguments or when no entry is usable.
+ */
+int tidar_pick_draft_length(const double *step_us, int n, double alpha, double *tokens_per_us);
+
+/*
+ * tidar_kv_commit over paged KV caches (see tidar_attn_step_paged for the
+ * layout).  k_pools / v_pools: device arrays of L device pointers, one pool
+ * [num_pages, Hkv, 64, D] per layer; block_table [B, max_pages] as for the
+ * attention.  The pages that receive rows P_b .. P_b + j* - 1 must already be
+ * in the block table (the caller allocates pages before the step); an invalid
+ * id there sets TIDAR_DEV_BAD_PAGE and leaves the sequence untouched.
+ * Everything else as tidar_kv_commit (same workspace size).
+ */
+tidar_status tidar_kv_commit_paged(void *const *k_pools, void *const *v_pools,
+                                   const void *const *k_news, const void *const *v_news,
+                                   const int32_t *block_table, int max_pages, int num_pages,
+                                   int L, int B, int Hkv, int D, int k,
+                                   int32_t *prefix_len, const int32_t *accept_len, const int32_t *resampled,
+                                   const void *group_logits, int logits_dtype, int V, const float *u_draft,
+                                   int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group,
+                                   void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *tidar_status_string(tidar_status s);

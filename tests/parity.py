@@ -15,10 +15,10 @@ import oracle
 EXEMPT = 1e-5
 
 
-def compare_verify(inp, got, report):
+def compare_verify(inp, got, report, trust_ar=1.0):
     """Checks the GPU verify outputs `got` against the oracle on `inp`; returns the oracle's outputs (with
     exempt decisions replaced by the GPU's)."""
-    ref = oracle.verify(inp)
+    ref = oracle.verify(inp, trust_ar=trust_ar)
     B, k = inp["drafts"].shape
     forced = np.full(B, -1, np.int32)
     for b in range(B):
@@ -29,7 +29,7 @@ def compare_verify(inp, got, report):
             report.append(("accept", b, margin))
             forced[b] = got["accept_len"][b]
     if (forced >= 0).any():
-        ref = oracle.verify(inp, forced_accept_len=forced)
+        ref = oracle.verify(inp, forced_accept_len=forced, trust_ar=trust_ar)
     assert np.array_equal(got["accept_len"], ref["accept_len"])
     for b in range(B):
         if got["resampled"][b] != ref["resampled"][b]:

@@ -31,7 +31,7 @@ def test_algorithmic_bytes_closed_form():
 
 def test_kernels_per_step():
     cfg = synth.CONFIGS["qwen3-8b_k8"]
-    assert bench.kernels_per_step(cfg) == cfg.L + 3  # L attention launches, verify (2), commit (1)
+    assert bench.kernels_per_step(cfg) == cfg.L + 2  # L attention launches, verify (1), commit (1)
 
 
 def test_clock_sample_parsing():
@@ -84,7 +84,7 @@ def test_reference_arm_line():
 
 
 def test_line_sanity_rules():
-    line = {"value": 1000.0, "ms_per_step": 1.0, "steps": 10, "gpu_launches": 390,
+    line = {"value": 1000.0, "ms_per_step": 1.0, "steps": 10, "gpu_launches": 380,
             "roofline": {"us_per_launch": 20.0}, "e2e": {"value": 500.0}}
     bench.check_line(line)
     with pytest.raises(AssertionError):  # end to end cannot beat the device-only rate

@@ -57,6 +57,36 @@ def test_verify_many_small_cases():
     assert len(report) <= 2
 
 
+@pytest.mark.parametrize("trust_ar", [0.0, 0.37, 0.8, 1.0])
+@pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k16", "qwen3-8b_k8_b8"])
+def test_verify_trust_mix_parity(name, trust_ar):
+    """tidar_verify_trust_mix against the oracle's mixed target softmax(lambda z_AR + (1 - lambda) z_diff)."""
+    cfg = synth.CONFIGS[name]
+    report = []
+    for seed in range(2):
+        inp = synth.make_verify_inputs(cfg, seed=seed)
+        got = _gpu().verify(inp, trust_ar=trust_ar)
+        compare_verify(inp, got, report, trust_ar=trust_ar)
+        if trust_ar == 0.0:
+            assert (got["accept_len"] == cfg.k).all()
+    print(f"{name} lambda={trust_ar}: exemptions {report}")
+    assert len(report) <= 1
+
+
+def test_verify_trust_mix_many_small_cases():
+    """Small vocabularies, many sequences: the mixed target moves accept lengths across 0..k."""
+    report = []
+    rng = np.random.default_rng(5)
+    for V, k, dtype, lam in ((8, 4, "f32", 0.5), (1000, 16, "f32", 0.25), (9000, 3, "bf16", 0.75)):
+        cfg = synth.CONFIGS["tiny"].with_(B=256, V=V, k=k, logits_dtype=dtype, cfg_id=200 + V)
+        inp = synth.make_verify_inputs(cfg, seed=int(rng.integers(1 << 30)))
+        got = _gpu().verify(inp, trust_ar=lam)
+        compare_verify(inp, got, report, trust_ar=lam)
+        assert len(set(got["accept_len"].tolist())) > 1
+    print(f"exemptions {report}")
+    assert len(report) <= 2
+
+
 def test_verify_bad_draft_sets_status():
     cfg = synth.CONFIGS["tiny"].with_(B=2)
     inp = synth.make_verify_inputs(cfg, seed=1)

@@ -55,7 +55,8 @@ def attn(inp: dict, Hq: int, Hkv: int, D: int, k: int, mode: int = abi.TIDAR_MAS
     return res
 
 
-def verify(inp: dict, want_status=False):
+def verify(inp: dict, want_status=False, trust_ar=None):
+    """tidar_verify on the numpy inputs (tidar_verify_trust_mix when trust_ar is given)."""
     p, dt = logits_dev(inp["p_logits"])
     q, _ = logits_dev(inp["q_logits"])
     B, k, V = inp["p_logits"].shape
@@ -67,10 +68,14 @@ def verify(inp: dict, want_status=False):
                 logq_d=torch.zeros((B, k), dtype=torch.float32, device=DEV))
     ws = workspace(abi.tidar_verify_workspace_size(B, k, V))
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    abi.tidar_verify(p, q, dt, to_dev(inp["drafts"].astype(np.int32)), to_dev(inp["preaccepted"].astype(np.uint8)),
-                     to_dev(inp["u_acc"].astype(np.float32)), to_dev(inp["u_res"].astype(np.float32)), B, k, V,
-                     outs["accept_len"], outs["resampled"], outs["tokens"], outs["n_emitted"], outs["logp_d"],
-                     outs["logq_d"], ws, ws.numel(), st)
+    args = (p, q, dt, to_dev(inp["drafts"].astype(np.int32)), to_dev(inp["preaccepted"].astype(np.uint8)),
+            to_dev(inp["u_acc"].astype(np.float32)), to_dev(inp["u_res"].astype(np.float32)), B, k, V)
+    rest = (outs["accept_len"], outs["resampled"], outs["tokens"], outs["n_emitted"], outs["logp_d"],
+            outs["logq_d"], ws, ws.numel(), st)
+    if trust_ar is None:
+        abi.tidar_verify(*args, *rest)
+    else:
+        abi.tidar_verify_trust_mix(*args, trust_ar, *rest)
     torch.cuda.synchronize()
     res = {n: t.cpu().numpy() for n, t in outs.items()}
     if want_status:
