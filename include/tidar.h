@@ -152,7 +152,7 @@ tidar_status tidar_attn_step_paged(const void *q, const void *k_new, const void 
  * prefix_len int32 [B] (device)
  * theta      rotary base, > 1
  * q          bf16 [B, R, Hq, D]; k_new, v_new bf16 [B, R, Hkv, D]
- * D in {64, 128}, Hq % Hkv == 0, k in 1..16; all tensors 16-byte aligned.
+ * D in {64, 128}, Hq % Hkv == 0, k in 1..16; all tensors 4-byte aligned.
  * dev_status TIDAR_DEV_BAD_PREFIX (and that sequence's Q/K left unwritten) for
  *            a negative prefix length.
  */
