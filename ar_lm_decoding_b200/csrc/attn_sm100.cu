@@ -2,47 +2,48 @@
 //
 // One CTA owns 128 packed query rows (row m = r*G + g of the G query heads
 // sharing KV head kvh: GQA packing, so every K/V byte feeds 128 rows) and a
-// contiguous run of 64-key tiles of one sequence.  A sequence's tiles are
-// the cached prefix in 64-row tiles (the last one partial) followed by the
-// R new keys of this step in 64-row tiles.
+// contiguous run of 128-key tiles of one sequence.  A sequence's tiles are
+// the cached prefix in 128-row tiles (the last one partial) followed by the
+// R new keys of this step in 128-row tiles.
 //
 // Warp roles (12 warps):
 //   warps 0, 2  TMA producers of K and of V (128-byte swizzle), each into its
-//               own 4-stage ring: prefix tiles from the cache, new-key tiles
-//               from K_new/V_new through a 3-D tensor map (no head gather).
-//               A K stage is freed when its QK^T completes, a V stage when
-//               its PV does, so K runs ahead of V.
+//               own 3-stage ring: prefix tiles from the cache (two 64-row
+//               boxes per tile: with a paged cache each box is one page), new-
+//               key tiles from K_new/V_new through a 3-D tensor map (no head
+//               gather).  A K stage is freed when its QK^T completes, a V
+//               stage when its PV does, so K runs ahead of V.
 //   warp 1      TMEM owner; one thread issues S = Q K^T (tcgen05.mma, both
-//               operands in shared memory) into S buffer i % 4.
-//   warp 3      one thread issues O_w += P V with P read from TMEM (A operand
+//               operands in shared memory) into S buffer j % 3.
+//   warp 3      one thread issues O += P V with P read from TMEM (A operand
 //               in TMEM, V an MN-major operand in shared memory).
-//   warps 4-11  softmax, two warpgroups that take alternate key tiles:
-//               warpgroup w owns tiles i = w, w+2, w+4, ... of the CTA's run,
-//               S buffers w and w+2 (double buffered: the S of its next tile
-//               is computed while it works on this one) and its own
-//               accumulator O_w.  Thread = query row = TMEM lane, so each
-//               thread holds the whole row of its tile (64 scores in
-//               registers): the row max first, then the exponentials; the
-//               running max only moves (and O_w is rescaled) when the tile
-//               max exceeds it by more than 2^8, so p <= 2^8 always fits.  The
-//               two warpgroups never wait for each other.  The mask is
-//               evaluated from indices.
+//   warps 4-11  softmax: both warpgroups work on every tile, warpgroup w on
+//               its columns [64w, 64w+64); thread = query row = TMEM lane.
+//               The two halves of a row always hold the same running max,
+//               so their exponentials share a scale and PV sums them into
+//               the one O.  A tile is exponentiated against that (possibly
+//               stale) max -- exact as long as p <= 2^8 fits -- while its row
+//               max is taken in the same pass; the halves then exchange
+//               maxima through shared memory, and only rows whose max grew
+//               by more than 2^8 redo their exponentials and rescale O.  The
+//               mask is evaluated from indices.
 //   warps 2-11  also load Q when its rows cannot come through TMA.
-// TMEM (512 columns): S buffers at [64 j, 64 j + 64), j = 0..3; O_0 at
-// [256, 256+D), O_1 at [384, 384+D).  P (bf16) overwrites the first 32
-// columns of its S buffer.  QK(i) reuses the buffer that PV(i-4) reads and is
-// issued once PV(i-4) has completed.
-// At the end the two accumulators of a row are merged with the weights of
-// their running maxima (each warpgroup takes half of the columns), giving one
+// TMEM (512 columns): S buffers at [0, 128), [128, 256), [256, 384); O at
+// [384, 384+D).  P (bf16) overwrites the first 64 columns of its S buffer.
+// QK(j) reuses the buffer that PV(j-3) reads and is issued once PV(j-3) has
+// completed, so the softmax always has the next two tiles' S ready.
+// At the end each warpgroup reads its half of the columns of O and forms one
 // normalised partial row per query row, stored as fp16 with a per-half-row
 // fp32 scale (|error| <= 2^-12 of the row maximum) and its log2 LSE in fp32.
 // With one split that row is the output.  Otherwise the CTAs that split one
-// row tile's keys form a thread-block cluster: the records are pushed over
-// distributed shared memory into the idle K/V ring of the cluster CTA that
-// owns the row (a split cluster barrier: arrive once the ring is idle, wait
-// before pushing); after a second cluster barrier each CTA merges its slice
-// of rows over the S partials (LSE weights, fixed order) and writes the final
-// bf16 output and LSE.
+// row tile's keys form a thread-block cluster: each CTA stages its records in
+// its own (idle) K/V ring, in the layout of the block every owner receives,
+// and sends each owner its block with one shared-to-shared bulk copy that
+// counts the bytes on the owner's receive barrier (armed at set-up); every
+// CTA merges its slice of rows over the S blocks (LSE weights, fixed order)
+// as soon as they have all landed, and writes the final bf16 output and LSE.
+// The cluster barrier has two phases: every CTA's ring is idle (waited for
+// before sending), and every CTA has received its blocks (before exit).
 //
 // Before the previous kernel in the stream has finished (programmatic
 // dependent launch), a CTA sets up its barriers and TMEM and asks L2 for the
@@ -53,8 +54,8 @@
 // TIDAR_DEV_TIMEOUT in dev_status and every role stops; then the producers
 // wait for their copies in flight and the MMA issuers for their MMAs (bounded
 // waits that ignore the abort), so nothing lands in shared memory or TMEM
-// after the CTA frees it.  No wait sits between two CTA barriers that an
-// aborted warp could skip.
+// after the CTA frees it.  The softmax warps pass the per-tile named barrier
+// on every tile even after an abort, so no warp waits there for one that left.
 #include "attn.cuh"
 #include "tc.cuh"
 
@@ -63,14 +64,31 @@ namespace tidar {
 namespace {
 
 constexpr int TM = 128;
-constexpr int TN = 64;
-constexpr int STAGES = 4;
-constexpr int NSB = 4;  // S buffers: warpgroup w owns buffers w and w + 2
-static_assert(TN == kPageRows, "a KV-cache page is one key tile");
+constexpr int TN = 128;
+constexpr int BOXR = 64;  // rows of one TMA box of a paged cache (one page): a tile is two boxes
+constexpr int STAGES = 3;
 constexpr int THREADS = 384;
 constexpr int kMaxSplits = 8;                        // cluster size limit (portable clusters)
-constexpr int kPageSlots = kMaxPagesPerSeq + kMaxSplits;  // page ids of one CTA's run of cache tiles
 constexpr long long kDrainCycles = kAttnWaitCycles;  // bound of the waits that drain issued work
+static_assert(BOXR == kPageRows, "a TMA box of the cache is one page");
+
+// Split-KV exchange of an S-CTA cluster.  CTA s merges rows [s*per, (s+1)*per) of the row tile, per =
+// ceil(128 / S).  Every CTA sends each owner one block with its partial records of the owner's rows:
+//   vals [D/8][pv]  16-byte chunks (8 fp16 of one row, divided by the half-row scale), pv = per rounded up to an
+//                   odd number, so that reading one chunk of consecutive rows and reading the consecutive chunks
+//                   of one row both spread over all shared-memory banks
+//   hdr  [per]      float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
+// The owner receives the S blocks in source order.  Both the received blocks and the staged outgoing ones live
+// in the CTA's K/V ring, which is idle by then: [row statistics | received | staged].
+__host__ __device__ constexpr int xchg_per(int S) { return (TM + S - 1) / S; }
+__host__ __device__ constexpr int xchg_vals_bytes(int S, int D) { return (D / 8) * (xchg_per(S) | 1) * 16; }
+__host__ __device__ constexpr int xchg_block_bytes(int S, int D) { return xchg_vals_bytes(S, D) + xchg_per(S) * 16; }
+constexpr int xchg_region_max(int D) {
+    int m = 0;
+    for (int S = 2; S <= kMaxSplits; ++S) m = S * xchg_block_bytes(S, D) > m ? S * xchg_block_bytes(S, D) : m;
+    return (m + 127) / 128 * 128;
+}
+constexpr int kStatsBytes = 4 * TM * 4;  // row statistics exchanged between the warpgroups (start of the ring)
 
 template <int D>
 struct Smem {
@@ -78,30 +96,29 @@ struct Smem {
     static constexpr int KV_TILE = TN * D * 2;  // one of K or V
     static constexpr int STAGE = 2 * KV_TILE;
     static constexpr int KV_OFF = Q_BYTES;
+    static constexpr int RECV_OFF = KV_OFF + kStatsBytes;          // received blocks (inside the idle ring)
+    static constexpr int STAGE_OFF = RECV_OFF + xchg_region_max(D);  // staged outgoing blocks (idem)
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
-    // k_full, k_empty, v_full, v_empty, s_full[4], p_full[4], pv_done[4], o_final, q_full, fin_qk, fin_pv, stall
-    static constexpr int NBARS = 4 * STAGES + 3 * NSB + 5;
+    // k_full, k_empty, v_full, v_empty, s_full[3], p_full[3], pv_done[2], o_final, q_full, fin_qk, fin_pv, stall,
+    // recv
+    static constexpr int NBARS = 4 * STAGES + 14;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
-    static constexpr int PAGES_OFF = MISC_OFF + 16;  // page ids of the CTA's cache tiles (paged caches)
-    static constexpr int TOTAL = PAGES_OFF + kPageSlots * 4;
+    static constexpr int XM_OFF = MISC_OFF + 16;  // row-max exchange between the warpgroups: [2][2][TM] bf16
+    static constexpr int TOTAL = XM_OFF + 2 * 2 * TM * 2;
     static constexpr int ALLOC = TOTAL + 1024;  // alignment slack
 };
 
 static_assert(Smem<64>::ALLOC <= 227 * 1024 && Smem<128>::ALLOC <= 227 * 1024, "shared memory beyond 227 KB");
-
-// Bytes the split-KV exchange of an S-CTA cluster uses at the start of a CTA's (idle) K/V ring: the row
-// statistics, the S partial records of its rows (row stride rounded up to an odd number of chunks) and their
-// headers.
-constexpr int xchg_bytes(int S, int D) {
-    const int per = (TM + S - 1) / S;
-    return 4 * TM * 4 + S * (per | 1) * 2 * D + S * per * 16;
-}
-constexpr bool xchg_fits(int D) {
+static_assert(Smem<64>::STAGE_OFF + xchg_region_max(64) <= Smem<64>::BAR_OFF &&
+                  Smem<128>::STAGE_OFF + xchg_region_max(128) <= Smem<128>::BAR_OFF,
+              "split-KV exchange larger than the K/V ring");
+// the merge's per-row weights fit the row-statistics area: per rows x (S weights x 2 halves + 2)
+constexpr bool weights_fit() {
     for (int S = 2; S <= kMaxSplits; ++S)
-        if (xchg_bytes(S, D) > STAGES * 2 * TN * D * 2) return false;  // the K and V rings
+        if (xchg_per(S) * (2 * S + 2) * 4 > kStatsBytes) return false;
     return true;
 }
-static_assert(xchg_fits(64) && xchg_fits(128), "split-KV exchange larger than the K/V ring");
+static_assert(weights_fit(), "merge weights larger than the row-statistics area");
 
 // Bit i set iff key base+i lies in [a, b) (i = 0..31).
 __device__ __forceinline__ uint32_t range_bits(int a, int b, int base) {
@@ -132,9 +149,8 @@ __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv
     for (int kk = 0; kk < TN / 16; ++kk) tc::mma_ts(d_o, a_p + kk * 8, dv + kk * 128, id, (acc || kk > 0) ? 1u : 0u);
 }
 
-// Loads 64 raw scores (TMEM columns col .. col+63 of this thread's lane, keys kbase .. kbase+63 of the tile)
-// into x.  MASKED: only keys in [0, lo) and [glo, ghi) are kept; the others (garbage past the sequence
-// included) become -inf.
+// Loads this thread's 64 raw scores (TMEM columns col .. col+63 of its lane) into x.  MASKED: only keys
+// kbase + j in [0, lo) and [glo, ghi) are kept; the others (garbage past the sequence included) become -inf.
 template <bool MASKED>
 __device__ __forceinline__ void half_load(uint32_t col, int kbase, int lo, int glo, int ghi, float (&x)[64]) {
 #pragma unroll
@@ -156,14 +172,6 @@ __device__ __forceinline__ void half_load(uint32_t col, int kbase, int lo, int g
     }
 }
 
-__device__ __forceinline__ void load_scores(bool masked, uint32_t col, int kbase, int lo, int glo, int ghi,
-                                            float (&x)[64]) {
-    if (masked)
-        half_load<true>(col, kbase, lo, glo, ghi, x);
-    else
-        half_load<false>(col, kbase, lo, glo, ghi, x);
-}
-
 __device__ __forceinline__ float half_max(const float (&x)[64]) {
     float m8[8];  // eight independent chains
 #pragma unroll
@@ -174,71 +182,75 @@ __device__ __forceinline__ float half_max(const float (&x)[64]) {
 }
 
 // p = 2^(x * sl2 + neg_m) for the 64 scores in x (-inf gives exactly 0), written as 32 bf16 pairs to TMEM
-// columns pcol .. pcol+31 (P, the A operand of PV).  Returns the sum of the 64 values of p.
-__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], float sl2, float neg_m) {
-    float sum8[8];
+// columns pcol .. pcol+31 (P, the A operand of PV).  Returns the sum of the 64 values of p; *mx receives the
+// maximum of x, computed in the same pass (its ALU work hides under the exponentials).
+__device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], float sl2, float neg_m, float *mx) {
+    float sum8[8], m8[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sum8[j] = 0.f;
+    for (int j = 0; j < 8; ++j) {
+        sum8[j] = 0.f;
+        m8[j] = -INFINITY;
+    }
     uint32_t pk[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const float a = fast_exp2(fmaf(x[2 * j], sl2, neg_m));
         const float bb = fast_exp2(fmaf(x[2 * j + 1], sl2, neg_m));
+        m8[(2 * j) & 7] = fmaxf(m8[(2 * j) & 7], x[2 * j]);
+        m8[(2 * j + 1) & 7] = fmaxf(m8[(2 * j + 1) & 7], x[2 * j + 1]);
         sum8[(2 * j) & 7] += a;
         sum8[(2 * j + 1) & 7] += bb;
         pk[j] = pack_bf16x2(a, bb);
     }
     tc::tmem_st32(pcol, pk);
+    *mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
     return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 }
 
-// Shared-memory layout of the split-KV exchange inside a CTA's (idle) K/V ring.  CTA s of an S-CTA cluster
-// merges rows [s*per, (s+1)*per) of the row tile, per = ceil(128 / S):
-//   [0, 4*TM floats)    row statistics exchanged between the warpgroups
-//   vals [S][D/8][pv]   16-byte chunks (8 fp16 of one row, divided by the half-row scale); pv = per rounded up
-//                       to an odd number, so that reading one chunk of consecutive rows and reading the
-//                       consecutive chunks of one row both spread over all shared-memory banks
-//   hdr  [S][per]       float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
-template <int D>
-struct Xchg {
-    uint8_t *base;
-    int S, per, pv;
-    __device__ Xchg(uint8_t *ring, int S_, int per_)
-        : base(ring + 4 * TM * sizeof(float)), S(S_), per(per_), pv(per_ | 1) {}
-    __device__ uint4 *vals() const { return reinterpret_cast<uint4 *>(base); }
-    __device__ float4 *hdr() const { return reinterpret_cast<float4 *>(base + (size_t)S * pv * 2 * D); }
-};
-
-// Merge of this CTA's rows over the S partial records of its cluster (all THREADS threads): item = (row,
-// 16-byte column chunk), consecutive threads on consecutive chunks of one row, so that every warp writes whole
-// output rows; each item weighs the S chunks by exp2(lse_s - max) * scale_s / sum.
+// Merge of this CTA's rows over the S blocks received (all THREADS threads).  First the weights of every row:
+// w_s = exp2(lse_s - max) / sum * scale_s per column half (in the row-statistics area, free by then); then items
+// (row, 16-byte column chunk), consecutive threads on consecutive chunks of one row, so that every warp writes
+// whole output rows.  Sources are summed in a fixed order.
 template <int D, int S>
-__device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, int split, int mt, int b, int kvh,
-                                           int tid) {
-    constexpr int per = (TM + S - 1) / S, CH = D / 8;
-    const Xchg<D> x(ring, S, per);
+__device__ __forceinline__ void merge_rows(const AttnParams &p, const uint8_t *recv, float *wts, int split, int mt,
+                                           int b, int kvh, int tid) {
+    constexpr int per = xchg_per(S), pv = per | 1, CH = D / 8, VB = xchg_vals_bytes(S, D), BB = xchg_block_bytes(S, D);
     const int row0 = split * per, nrows = max(0, min(TM, row0 + per) - row0);
-    for (int it = tid; it < nrows * CH; it += THREADS) {
-        const int rl = it / CH, c = it - rl * CH;
+    for (int rl = tid; rl < nrows; rl += THREADS) {
         float4 hd[S];
-        uint4 raw[S];
-#pragma unroll
-        for (int sp = 0; sp < S; ++sp) {
-            hd[sp] = x.hdr()[sp * per + rl];
-            raw[sp] = x.vals()[(sp * CH + c) * x.pv + rl];
-        }
         float mx = -INFINITY;
 #pragma unroll
-        for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, hd[sp].x);
-        float acc[8], wsum = 0.f;
+        for (int sp = 0; sp < S; ++sp) {
+            hd[sp] = reinterpret_cast<const float4 *>(recv + sp * BB + VB)[rl];
+            mx = fmaxf(mx, hd[sp].x);
+        }
+        float wq[S], wsum = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) {
+            wq[sp] = hd[sp].x == -INFINITY ? 0.f : fast_exp2(hd[sp].x - mx);
+            wsum += wq[sp];
+        }
+        const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+        float *w = wts + rl * (2 * S + 2);
+#pragma unroll
+        for (int sp = 0; sp < S; ++sp) {
+            w[2 * sp] = wq[sp] * winv * hd[sp].y;
+            w[2 * sp + 1] = wq[sp] * winv * hd[sp].z;
+        }
+        w[2 * S] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;  // natural-log LSE
+    }
+    __syncthreads();
+    for (int it = tid; it < nrows * CH; it += THREADS) {
+        const int rl = it / CH, c = it - rl * CH;
+        const float *w = wts + rl * (2 * S + 2);
+        float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int sp = 0; sp < S; ++sp) {
-            const float wq = hd[sp].x == -INFINITY ? 0.f : fast_exp2(hd[sp].x - mx);
-            wsum += wq;
-            const float f = wq * (c < CH / 2 ? hd[sp].y : hd[sp].z);
-            const uint32_t u[4] = {raw[sp].x, raw[sp].y, raw[sp].z, raw[sp].w};
+            const uint4 raw = reinterpret_cast<const uint4 *>(recv + sp * BB)[c * pv + rl];
+            const float f = w[2 * sp + (c < CH / 2 ? 0 : 1)];
+            const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 v = unpack_half2(u[e]);
@@ -248,13 +260,12 @@ __device__ __forceinline__ void merge_rows(const AttnParams &p, uint8_t *ring, i
         }
         const int m = mt * TM + row0 + rl;
         if (m < p.M) {
-            const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
             const int rq = m / p.G;
             const size_t orow = (size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G);
             *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) =
-                make_uint4(pack_bf16x2(acc[0] * winv, acc[1] * winv), pack_bf16x2(acc[2] * winv, acc[3] * winv),
-                           pack_bf16x2(acc[4] * winv, acc[5] * winv), pack_bf16x2(acc[6] * winv, acc[7] * winv));
-            if (c == 0 && p.lse) p.lse[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                           pack_bf16x2(acc[6], acc[7]));
+            if (c == 0 && p.lse) p.lse[orow] = w[2 * S];
         }
     }
 }
@@ -288,16 +299,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto k_empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto v_full = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
     auto v_empty = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
-    // Per S buffer sb = i % 4 (tile i is its (i / 4)-th use and completes phase i / 4 of each):
-    auto s_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + sb); };           // S(i) is in buffer sb
-    auto p_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + NSB + sb); };     // P(i) is in buffer sb
-    auto pv_done = [&](int sb) { return bar0 + 8u * (4 * STAGES + 2 * NSB + sb); }; // PV(i) has completed
-    constexpr int X = 4 * STAGES + 3 * NSB;
-    const uint32_t o_final = bar0 + 8u * X;        // one phase: the last PV has completed
-    const uint32_t q_full = bar0 + 8u * (X + 1);
-    const uint32_t fin_qk = bar0 + 8u * (X + 2);   // the QK issuer's MMAs have all completed
-    const uint32_t fin_pv = bar0 + 8u * (X + 3);   // the PV issuer's MMAs have all completed
-    const uint32_t stall = bar0 + 8u * (X + 4);    // nothing arrives here (timeout test)
+    auto s_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + sb); };      // S buffer sb holds a new S
+    auto p_full = [&](int sb) { return bar0 + 8u * (4 * STAGES + 3 + sb); };  // P in S buffer sb is complete
+    // pv_done(e): its k-th phase completes with PV(2k + e).  Waiting for PV(i) on pv_done(i & 1) is unambiguous
+    // once PV(i-2) has completed, which holds wherever it is waited for (see there).
+    auto pv_done = [&](int e) { return bar0 + 8u * (4 * STAGES + 6 + e); };
+    const uint32_t o_final = bar0 + 8u * (4 * STAGES + 8);  // one phase: the last PV has completed
+    const uint32_t q_full = bar0 + 8u * (4 * STAGES + 9);
+    const uint32_t fin_qk = bar0 + 8u * (4 * STAGES + 10);  // the QK issuer's MMAs have all completed
+    const uint32_t fin_pv = bar0 + 8u * (4 * STAGES + 11);  // the PV issuer's MMAs have all completed
+    const uint32_t stall = bar0 + 8u * (4 * STAGES + 12);   // nothing arrives here (timeout test)
+    const uint32_t recv = bar0 + 8u * (4 * STAGES + 13);    // every CTA's block of this CTA's rows has landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -305,6 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int b = bh / p.Hkv, kvh = bh % p.Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long wl = p.wait_cycles;
+    const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
     // ---- set-up that needs nothing from the previous kernel (programmatic dependent launch) ----
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -313,18 +326,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc::mbar_init(v_full(s), 1);
             tc::mbar_init(v_empty(s), 1);
         }
-        for (int sb = 0; sb < NSB; ++sb) {
+        for (int sb = 0; sb < 3; ++sb) {
             tc::mbar_init(s_full(sb), 1);
-            tc::mbar_init(p_full(sb), 128);  // the owning warpgroup's threads
-            tc::mbar_init(pv_done(sb), 1);
+            tc::mbar_init(p_full(sb), 256);  // both softmax warpgroups
         }
+        tc::mbar_init(pv_done(0), 1);
+        tc::mbar_init(pv_done(1), 1);
         tc::mbar_init(o_final, 1);
         tc::mbar_init(q_full, q_tma ? 1 : THREADS - 64);
         tc::mbar_init(fin_qk, 1);
         tc::mbar_init(fin_pv, 1);
         tc::mbar_init(stall, 1);
+        tc::mbar_init(recv, 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
+        // armed now with the bytes it is to receive (one block from every CTA of the cluster, itself included):
+        // its phase completes when the last block lands
+        if (S > 1) tc::mbar_arrive_expect_tx(recv, S * xchg_block_bytes(S, D));
         tc::tma_prefetch_desc(&tm_kc);
         tc::tma_prefetch_desc(&tm_vc);
         tc::tma_prefetch_desc(&tm_kn);
@@ -334,18 +352,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int P_hint = __ldcg(p.prefix_len + b);
         if (P_hint >= 0 && P_hint <= p.P_max) {
             int TPh, h0, h1;
-            split_range(P_hint, p.R, split, p.n_splits, TPh, h0, h1);
+            split_range(P_hint, p.R, split, S, TPh, h0, h1);
             for (int t = h0; t < min(h1, min(h0 + STAGES, TPh)); ++t) {
-                int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
-                if (p.block_table) {
-                    const int pg = __ldcg(p.block_table + (size_t)b * p.max_pages + t);
-                    if (pg < 0 || pg >= p.num_pages) break;
-                    y = (pg * p.Hkv + kvh) * TN;
-                }
+                for (int h2 = 0; h2 < (p.block_table ? 2 : 1); ++h2) {
+                    int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
+                    if (p.block_table) {
+                        if (2 * t + h2 >= p.max_pages) continue;
+                        const int pg = __ldcg(p.block_table + (size_t)b * p.max_pages + 2 * t + h2);
+                        if (pg < 0 || pg >= p.num_pages) continue;
+                        y = (pg * p.Hkv + kvh) * BOXR;
+                    }
 #pragma unroll
-                for (int h = 0; h < D / 64; ++h) {
-                    tc::tma_prefetch_l2_2d(&tm_kc, h * 64, y);
-                    tc::tma_prefetch_l2_2d(&tm_vc, h * 64, y);
+                    for (int h = 0; h < D / 64; ++h) {
+                        tc::tma_prefetch_l2_2d(&tm_kc, h * 64, y);
+                        tc::tma_prefetch_l2_2d(&tm_vc, h * 64, y);
+                    }
                 }
             }
         }
@@ -363,19 +384,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     const int P = p.prefix_len[b];
-    int TP, t0, t1;
+    int TP = 0, t0 = 0, t1 = 0;
     const bool bad_prefix = P < 0 || P > p.P_max;
-    if (!bad_prefix) split_range(P, p.R, split, p.n_splits, TP, t0, t1);
-    int *pages = reinterpret_cast<int *>(smem + L::PAGES_OFF);  // pages[i]: page of cache tile t0 + i
+    if (!bad_prefix) split_range(P, p.R, split, S, TP, t0, t1);
     bool bad_page = false;
     if (p.block_table && !bad_prefix) {  // (uniform over the CTA: one sequence)
         // every CTA of the cluster checks every page of the sequence, so that they all take the same exit (the
-        // early one below passes no cluster barrier); it keeps the ids of its own tiles
+        // early one below passes no cluster barrier)
         int bad = 0;
-        for (int t = tid; t < TP; t += THREADS) {
-            const int pg = p.block_table[(size_t)b * p.max_pages + t];
+        const int np = ceil_div(P, BOXR);  // pages holding rows [0, P)
+        const int32_t *row_pages = p.block_table + (size_t)b * p.max_pages;
+        for (int pi = tid; pi < np; pi += THREADS) {
+            const int pg = row_pages[pi];
             bad |= pg < 0 || pg >= p.num_pages;
-            if (t >= t0 && t < t1) pages[t - t0] = pg;
         }
         bad_page = __syncthreads_or(bad) != 0;
     }
@@ -392,16 +413,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
     const int n = t1 - t0;
+    // cache row of box h2 (0, 1: the two 64-row halves) of cache tile t: contiguous, or through the block table
+    // (read as the copy is issued; the table is not written during the launch).  The second box of a last tile
+    // that ends within its first page has no page of its own: it re-reads the first page (rows past P are
+    // excluded from the scores and their V rows zeroed).
+    auto cache_row = [&](int t, int h2) {
+        if (!p.block_table) return (b * p.Hkv + kvh) * p.P_max + t * TN + h2 * BOXR;
+        const int pi = 2 * t + h2;
+        const int pg = __ldcg(p.block_table + (size_t)b * p.max_pages + (pi < ceil_div(P, BOXR) ? pi : pi - 1));
+        return (pg * p.Hkv + kvh) * BOXR;
+    };
 
-    // K (is_v = 0) or V (is_v = 1) of tile i into stage i % STAGES of its ring
+    // K (is_v = 0) or V (is_v = 1) of tile i into stage i % STAGES of its ring: two 64-row boxes per column block
     auto issue_tile = [&](int i, int is_v) {
         const int st = i % STAGES;
         const uint32_t bar = is_v ? v_full(st) : k_full(st);
         tc::mbar_arrive_expect_tx(bar, L::KV_TILE);
         const int t = t0 + i;
         const uint32_t dst = sKV + st * L::STAGE + is_v * L::KV_TILE;
-        if (t < TP) {
-            const int y = p.block_table ? (pages[i] * p.Hkv + kvh) * TN : (b * p.Hkv + kvh) * p.P_max + t * TN;
+        if (t < TP && p.block_table) {  // two 64-row boxes, one per page
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int y = cache_row(t, h2);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                    tc::tma_load_2d(dst + h * TN * 128 + h2 * BOXR * 128, is_v ? &tm_vc : &tm_kc, h * 64, y, bar);
+            }
+        } else if (t < TP) {  // one 128-row box per column block
+            const int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
 #pragma unroll
             for (int h = 0; h < D / 64; ++h) tc::tma_load_2d(dst + h * TN * 128, is_v ? &tm_vc : &tm_kc, h * 64, y, bar);
         } else {
@@ -415,10 +454,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---- thread 0 starts the first copies at once ----
     const int prologue = min(n, STAGES);
     if (tid == 0) {
-        for (int i = 0; i < prologue; ++i) {
-            issue_tile(i, 0);
-            issue_tile(i, 1);
-        }
+        for (int i = 0; i < prologue; ++i) issue_tile(i, 0);
+        for (int i = 0; i < prologue; ++i) issue_tile(i, 1);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -447,8 +484,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp < 4) {
         if (warp == 0 || warp == 2) {
             // ================= TMA producers: warp 0 streams K, warp 2 streams V =================
-            // K of a tile is released as soon as its QK^T completes, V after its PV, so the K ring
-            // runs ahead of the V ring and QK^T of the next tiles never waits behind a PV.
             const int is_v = warp == 2;
             if (lane == 0) {
                 int issued = prologue;
@@ -467,8 +502,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!is_v && q_tma) tc::mbar_wait_drain(q_full, 0, kDrainCycles);
             }
             __syncwarp();
-        } else if (warp == 1 || warp == 3) {
+        } else {
             // ================= MMA issue: QK^T on warp 1, PV on warp 3 (one thread each) =================
+            // S of tile j goes to S buffer j % 3.  QK(j), j >= 3, reuses the buffer whose P PV(j-3) reads, so it
+            // is issued once PV(j-3) has completed; the softmax still has S(j-2) and S(j-1) to work on.
             constexpr uint64_t kStage = L::STAGE >> 4;  // one ring stage in the descriptor's address field
             const uint32_t tb = tbase;
             if (lane == 0 && warp == 1) {
@@ -481,16 +518,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ok = ok && tc::mbar_wait(q_full, 0, abort_flag, wl);
                 int kst = 0;
                 uint32_t kph = 0;
-                for (int i = 0; i < n && ok; ++i) {
-                    const int sb = i & (NSB - 1);
-                    if (i >= NSB) {  // PV(i-4) has read P out of S buffer sb
-                        ok = tc::mbar_wait(pv_done(sb), ((i >> 2) - 1) & 1, abort_flag, wl);
+                for (int j = 0; j < n && ok; ++j) {
+                    const int sb = j % 3;
+                    if (j >= 3) {  // PV(j-3) done reading P from buffer sb (PV(j-5) was waited for before)
+                        ok = tc::mbar_wait(pv_done((j - 3) & 1), ((j - 3) >> 1) & 1, abort_flag, wl);
                         if (!ok) break;
                     }
                     ok = tc::mbar_wait(k_full(kst), kph, abort_flag, wl);
                     if (!ok) break;
                     tc::fence_after_sync();
-                    issue_qk<D>(tb + sb * TN, dq, dk + kst * kStage, id_qk);
+                    issue_qk<D>(tb + sb * 128, dq, dk + kst * kStage, id_qk);
                     tc::mma_commit(s_full(sb));
                     tc::mma_commit(k_empty(kst));
                     if (++kst == STAGES) {
@@ -507,14 +544,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 int vst = 0;
                 uint32_t vph = 0;
                 for (int i = 0; i < n && ok; ++i) {
-                    const int sb = i & (NSB - 1), w = i & 1;
+                    const int sb = i % 3;
                     ok = tc::mbar_wait(v_full(vst), vph, abort_flag, wl) &&
-                         tc::mbar_wait(p_full(sb), (i >> 2) & 1, abort_flag, wl);
+                         tc::mbar_wait(p_full(sb), (i / 3) & 1, abort_flag, wl);
                     if (!ok) break;
                     tc::fence_after_sync();
-                    issue_pv<D>(tb + 256 + w * 128, tb + sb * TN, dv + vst * kStage, id_pv, i >= 2);
+                    issue_pv<D>(tb + 384, tb + sb * 128, dv + vst * kStage, id_pv, i > 0);
                     tc::mma_commit(v_empty(vst));
-                    tc::mma_commit(pv_done(sb));
+                    tc::mma_commit(pv_done(i & 1));
                     if (i == n - 1) tc::mma_commit(o_final);
                     if (++vst == STAGES) {
                         vst = 0;
@@ -526,26 +563,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
         __syncwarp();
-        // the cluster barrier's two phases: rings idle (records may be pushed), records pushed.  These warps
-        // publish nothing, so their arrivals carry no release fence.
+        // these warps are done with the ring (copies drained, MMAs complete): first phase of the cluster barrier
         tc::cluster_arrive_relaxed();
         tc::cluster_wait();
-        tc::cluster_arrive_relaxed();
-        tc::cluster_wait();
-        if (warp == 1) {
-            tc::fence_after_sync();
-            tc::tmem_dealloc(tbase, 512);
-        }
     } else {
-        // ================= softmax: warpgroup w on tiles i = w, w+2, ... =================
+        // ================= softmax: both warpgroups on every tile =================
+        // Warpgroup w takes columns [64w, 64w+64) of each S tile (thread = query row = TMEM lane).  The two
+        // halves of a row agree on one running max through a small exchange in shared memory, so both scale
+        // their exponentials alike and PV sums them into the one O accumulator.
         const int w = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const int m_row = mt * TM + row;
         const int r = m_row / p.G;
-        const int wt = tid - 128 - 128 * w;  // 0..127 within the warpgroup
-        // every row of this warp is padding of the last row tile: P = 0, no exponentials
-        const bool pad_warp = mt * TM + q4 * 32 >= p.M;
+        const int wt = tid - 128;  // 0..255
         // visible new keys of row r: [0, vis_lim) and [vis_glo, vis_ghi) (same rule as new_key_visible)
         int vis_lim, vis_glo = 0, vis_ghi = 0;
         if (p.mask_mode == TIDAR_MASK_CAUSAL || r < p.k) {
@@ -557,17 +588,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             vis_ghi = vis_glo + p.k;
         }
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-        const uint32_t o_col = tbase + lane_off + 256 + w * 128;  // O_w
+        const uint32_t o_col = tbase + lane_off + 384 + w * (D / 2);  // this warpgroup's half of O
+        __nv_bfloat16 *xm = reinterpret_cast<__nv_bfloat16 *>(smem + L::XM_OFF);  // [2 tiles][2 wg][TM]
         const float sl2 = p.scale_log2;  // > 0, so the max of raw scores gives the max of scaled ones
-        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units) and sum of this row's tiles
+        float m_run = -INFINITY, l_run = 0.f;  // running max (scaled log2 units, shared by both halves), own sum
         bool ok = true;
-        for (int i = w; i < n; i += 2) {
-            const int sb = i & (NSB - 1);
-            const uint32_t s_col = tbase + lane_off + sb * TN;  // S buffer of tile i
-            if (ok) ok = tc::mbar_wait(s_full(sb), (i >> 2) & 1, abort_flag, wl);
-            ok = __all_sync(0xffffffffu, ok);  // TMEM accesses are warp-collective: decide per warp
-            if (!ok) continue;                // nothing below waits on other threads: skipping is safe
-            tc::fence_after_sync();
+        for (int i = 0; i < n; ++i) {
+            const int sb = i % 3;
+            bool have = ok && tc::mbar_wait(s_full(sb), (i / 3) & 1, abort_flag, wl);
+            ok = __all_sync(0xffffffffu, have);  // TMEM accesses are warp-collective: decide per warp
+            const uint32_t s_col = tbase + lane_off + sb * 128;
             const int t = t0 + i;
             // a partial prefix tile (keys beyond P) or a new-key tile (the TiDAR mask): the visible keys of
             // this row are [0, lo) and [glo, ghi); everything else, garbage included, is excluded by select
@@ -587,54 +617,74 @@ __global__ void __launch_bounds__(THREADS, 1)
                 lo = min(lo, end);
                 ghi = min(ghi, end);
             }
-            if (pad_warp) {
-                uint32_t z[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) z[j] = 0u;
-                tc::tmem_st32(s_col, z);
-            } else {
-                float x[64];
-                load_scores(masked, s_col, 0, lo, glo, ghi, x);
-                const float mx = half_max(x) * sl2;  // the tile's row max
-                // the running max moves only when the tile's max exceeds it by more than 2^8 (always on the
-                // first tile with a visible key)
-                const bool grow = mx > m_run + 8.f;
-                if (__any_sync(0xffffffffu, grow)) {
-                    const float m_new = grow ? mx : m_run;
-                    const float f = grow ? fast_exp2(m_run - m_new) : 1.f;  // 0 when m_run = -inf
-                    if (i >= 2) {
-                        // rescale O_w, last written by PV(i-2) (complete: QK(i) was issued after PV(i-4), and
-                        // the wait below makes the order explicit)
-                        const int ip = i - 2;
-                        bool ok2 = tc::mbar_wait(pv_done(ip & (NSB - 1)), (ip >> 2) & 1, abort_flag, wl);
-                        ok = __all_sync(0xffffffffu, ok2);
-                        if (!ok) continue;
-                        tc::fence_after_sync();
+            float x[64];
+            const uint32_t pcol = s_col + w * 32;  // P of keys [64w, 64w+64) over S columns [32w, 32w+32)
+            const bool fresh = m_run == -INFINITY;  // no visible key so far: no max to reuse
+            float hmx = -INFINITY, lt = 0.f;
+            if (ok) {
+                tc::fence_after_sync();
+                if (masked)
+                    half_load<true>(s_col + w * 64, w * 64, lo, glo, ghi, x);
+                else
+                    half_load<false>(s_col + w * 64, w * 64, lo, glo, ghi, x);
+                // Exponentials against the running max the two halves already share (stale by design: exact as
+                // long as p <= 2^8); the tile's row max comes out of the same pass.  Only a row whose max grew by
+                // more than 2^8 -- all rows on the first tile, rarely later -- redoes them with the new max.
+                lt = fresh ? 0.f : half_exp(pcol, x, sl2, -m_run, &hmx);
+                if (fresh) hmx = half_max(x);
+            }
+            // both halves' maxima (rounded to bf16 for the exchange: any value the two sides agree on and that
+            // is within 2^8 of the true maximum serves); every warp passes this barrier on every tile
+            const __nv_bfloat16 hb = __float2bfloat16_rn(hmx);
+            xm[((i & 1) * 2 + w) * TM + row] = hb;
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");
+            const __nv_bfloat16 ob = xm[((i & 1) * 2 + (1 - w)) * TM + row];
+            if (ok) {
+                const float mx = fmaxf(__bfloat162float(hb), __bfloat162float(ob)) * sl2;
+                const float m_new = fmaxf(m_run, mx);
+                const bool grow = m_new > m_run + 8.f;
+                if (__any_sync(0xffffffffu, grow || fresh)) {  // fresh rows have written no P yet
+                    if (i >= 1 && __any_sync(0xffffffffu, grow)) {
+                        // rescale this half of O once PV(i-1), the last to write it, has completed.  S(i) is
+                        // complete, and QK(i) was issued after PV(i-3) completed: the wait below is unambiguous.
+                        const bool got =
+                            tc::mbar_wait(pv_done((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, wl);
+                        ok = __all_sync(0xffffffffu, got);
+                        if (ok) {
+                            tc::fence_after_sync();
+                            const float f = grow ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t v[32];
-                            tc::tmem_ld32(o_col + c * 32, v);
-                            tc::tmem_wait_ld();
+                            for (int c = 0; c < D / 64; ++c) {
+                                uint32_t v[32];
+                                tc::tmem_ld32(o_col + c * 32, v);
+                                tc::tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-                            tc::tmem_st32(o_col + c * 32, v);
+                                for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+                                tc::tmem_st32(o_col + c * 32, v);
+                            }
                         }
                     }
-                    l_run *= f;
-                    m_run = m_new;
+                    if (ok) {
+                        if (grow) {
+                            l_run *= fast_exp2(m_run - m_new);
+                            m_run = m_new;
+                        }
+                        tc::tmem_wait_st();  // the redone P overwrites the first pass's
+                        float unused;
+                        lt = half_exp(pcol, x, sl2, m_run == -INFINITY ? 0.f : -m_run, &unused);
+                    }
                 }
-                // exponentials: P of the tile's 64 keys goes to the first 32 columns of its S buffer
-                l_run += half_exp(s_col, x, sl2, m_run == -INFINITY ? 0.f : -m_run);
+                l_run += lt;
             }
             const int valid = tile_valid(t, TP, P, p.R);
-            if (valid < TN) {
+            if (ok && valid < TN) {
                 // keys past the sequence: zero their V rows (0 * garbage could be NaN) before PV reads them
                 const int st = i % STAGES;
-                bool ok2 = tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, wl);
-                ok = __all_sync(0xffffffffu, ok2);
+                const bool got = tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, wl);
+                ok = __all_sync(0xffffffffu, got);
                 if (ok) {
                     uint8_t *vrow = smem + L::KV_OFF + st * L::STAGE + L::KV_TILE;
-                    for (int idx = wt; idx < (TN - valid) * (D / 8); idx += 128) {
+                    for (int idx = wt; idx < (TN - valid) * (D / 8); idx += 256) {
                         const int j = valid + idx / (D / 8), c = idx % (D / 8);
                         *reinterpret_cast<uint4 *>(vrow + (c >> 3) * TN * 128 + j * 128 + ((c & 7) << 4)) =
                             make_uint4(0, 0, 0, 0);
@@ -653,46 +703,28 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool fin = ok && n > 0 && tc::mbar_wait(o_final, 0, abort_flag, wl);  // O final
         fin = __all_sync(0xffffffffu, fin);
         tc::fence_after_sync();
-        // this CTA's K/V ring is idle: once every CTA of the cluster has arrived here, the others may write
-        // their partial records into it (the wait is just before the push below).  The arrival publishes
-        // nothing, so it carries no release fence.
+        // this CTA's ring is idle (every PV has read its V): first phase of the cluster barrier
         tc::cluster_arrive_relaxed();
-        // the two accumulators of a row: O = (2^(m_0 - m) O_0 + 2^(m_1 - m) O_1) / l, l = the weighted sums
-        float *xs = reinterpret_cast<float *>(smem + L::KV_OFF);  // [4][TM]: m_0, l_0, m_1, l_1
-        xs[(2 * w) * TM + row] = m_run;
-        xs[(2 * w + 1) * TM + row] = l_run;
+        // the row sum is split over the two halves
+        float *xl = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM] in the row-statistics area
+        xl[w * TM + row] = l_run;
         asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        const float m0 = xs[row], l0 = xs[TM + row], m1 = xs[2 * TM + row], l1 = xs[3 * TM + row];
-        const float mm = fmaxf(m0, m1);
-        const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mm);
-        const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mm);
-        const float lt = a0 * l0 + a1 * l1;
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        const float lse2 = lt > 0.f ? mm + __log2f(lt) : -INFINITY;  // log2 of this CTA's row sum
-        const bool has1 = n >= 2;  // O_1 was written only if warpgroup 1 had a tile
-        const float f0 = a0 * inv, f1 = has1 ? a1 * inv : 0.f;
-        float hv[H];
+        const float ltot = l_run + xl[(1 - w) * TM + row];
+        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+        const float lse2 = ltot > 0.f ? m_run + __log2f(ltot) : -INFINITY;  // log2 of this CTA's row sum
+        uint32_t va[H / 32][32];
 #pragma unroll
         for (int c = 0; c < H / 32; ++c) {
-            uint32_t v0[32], v1[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v0[j] = v1[j] = 0u;
-            const uint32_t col = tbase + lane_off + 256 + w * H + c * 32;  // this warpgroup's half of the columns
-            if (fin) tc::tmem_ld32(col, v0);
-            if (fin && has1) tc::tmem_ld32(col + 128, v1);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                hv[c * 32 + j] = fin ? f0 * __uint_as_float(v0[j]) + (has1 ? f1 * __uint_as_float(v1[j]) : 0.f) : 0.f;
+            for (int j = 0; j < 32; ++j) va[c][j] = 0u;
+            if (fin) tc::tmem_ld32(o_col + c * 32, va[c]);
         }
-        const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
-        // CTA s of the cluster merges rows [s*per, (s+1)*per) of the tile; it receives every CTA's partial
-        // record of those rows in its (idle) ring: vals [S][D/8][per] 16-byte chunks (8 fp16 of one row),
-        // then hdr [S][per] float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
-        const int per = ceil_div(TM, S);
-        const Xchg<D> xc(smem + L::KV_OFF, S, per);
-        uint4 pk[H / 8];
-        float scale = 1.f;
+        tc::tmem_wait_ld();
+        float hv[H];
+#pragma unroll
+        for (int c = 0; c < H / 32; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) hv[c * 32 + j] = fin ? __uint_as_float(va[c][j]) * inv : 0.f;
         if (S == 1) {  // the CTA saw every key of its rows: the normalised half row is the output
             if (m_row < p.M) {
                 const size_t orow = (size_t)(b * p.R + r) * p.Hq + kvh * p.G + (m_row - r * p.G);
@@ -703,43 +735,64 @@ __global__ void __launch_bounds__(THREADS, 1)
                                         pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
                 if (w == 0 && p.lse) p.lse[orow] = lse2 * kLn2;
             }
+            tc::cluster_wait();  // (first phase)
         } else {
+            // this row's record, staged in this CTA's (idle) ring in the layout of the block its owner receives
             float am[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
             for (int j = 0; j < H; ++j) am[j & 3] = fmaxf(am[j & 3], fabsf(hv[j]));
             const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-            scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
+            const float scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
             const float rs = 1.f / scale;
+            const int per = xchg_per(S), pv = per | 1;
+            const int VB = xchg_vals_bytes(S, D), BB = xchg_block_bytes(S, D);
+            const int owner = row / per, rl = row - owner * per;
+            uint8_t *stage = smem + L::STAGE_OFF;  // [owner][vals | hdr]
+            uint4 *vals = reinterpret_cast<uint4 *>(stage + owner * BB);
 #pragma unroll
             for (int j = 0; j < H / 8; ++j)
-                pk[j] = make_uint4(pack_half2(hv[8 * j] * rs, hv[8 * j + 1] * rs), pack_half2(hv[8 * j + 2] * rs, hv[8 * j + 3] * rs),
-                                   pack_half2(hv[8 * j + 4] * rs, hv[8 * j + 5] * rs), pack_half2(hv[8 * j + 6] * rs, hv[8 * j + 7] * rs));
+                vals[(w * (H / 8) + j) * pv + rl] =
+                    make_uint4(pack_half2(hv[8 * j] * rs, hv[8 * j + 1] * rs), pack_half2(hv[8 * j + 2] * rs, hv[8 * j + 3] * rs),
+                               pack_half2(hv[8 * j + 4] * rs, hv[8 * j + 5] * rs), pack_half2(hv[8 * j + 6] * rs, hv[8 * j + 7] * rs));
+            float *hdr = reinterpret_cast<float *>(stage + owner * BB + VB) + rl * 4;
+            hdr[1 + w] = scale;
+            if (w == 0) hdr[0] = lse2;
+            tc::fence_proxy_async_smem();  // the bulk copies below read the staged records through the async proxy
+            asm volatile("bar.sync 1, 256;\n" ::: "memory");
+            tc::cluster_wait();  // every CTA's ring is idle: the blocks may land
+            if (tid == 128) {  // one block to every owner, this CTA included: it lands as source `split`
+                for (int o = 0; o < S; ++o)
+                    tc::bulk_copy_s2c(tc::cluster_map(sbase + L::RECV_OFF + split * BB, o), smem_u32(stage + o * BB),
+                                      BB, tc::cluster_map(recv, o));
+            }
         }
-        tc::cluster_wait();  // every CTA's ring is idle
-        if (S > 1) {  // push this row's record to the CTA that merges it (consecutive lanes: consecutive chunks)
-            const int owner = row / per, rl = row - owner * per;
-            const uint32_t ra =
-                tc::cluster_map(smem_u32(xc.vals() + ((size_t)split * (D / 8) + w * (H / 8)) * xc.pv + rl), owner);
-#pragma unroll
-            for (int j = 0; j < H / 8; ++j) tc::st_cluster_u32x4(ra + j * xc.pv * 16, pk[j]);
-            const uint32_t ha = tc::cluster_map(smem_u32(xc.hdr() + (size_t)split * per + rl), owner);
-            tc::st_cluster_f32(ha + 4 + 4 * w, scale);
-            if (w == 0) tc::st_cluster_f32(ha, lse2);
-        }
-        tc::fence_before_sync();
-        tc::cluster_sync();  // the records are in their owners' shared memory
     }
 
-    // ---- merge this CTA's rows over the cluster's S partial records (local shared memory, all threads) ----
-    switch (p.n_splits) {
-        case 2: merge_rows<D, 2>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        case 3: merge_rows<D, 3>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        case 4: merge_rows<D, 4>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        case 5: merge_rows<D, 5>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        case 6: merge_rows<D, 6>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        case 7: merge_rows<D, 7>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        case 8: merge_rows<D, 8>(p, smem + L::KV_OFF, split, mt, b, kvh, tid); break;
-        default: break;  // one split: each warpgroup wrote its half of every output row directly
+    // ---- merge this CTA's rows over the S blocks received (all threads), once they have all landed ----
+    if (S > 1) {
+        const bool got = tc::mbar_wait_drain(recv, 0, kDrainCycles);
+        if (!got && tid == 0) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
+        if (__syncthreads_and(got)) {
+            const uint8_t *rv = smem + L::RECV_OFF;
+            float *wts = reinterpret_cast<float *>(smem + L::KV_OFF);  // row-statistics area, free by now
+            switch (S) {
+                case 2: merge_rows<D, 2>(p, rv, wts, split, mt, b, kvh, tid); break;
+                case 3: merge_rows<D, 3>(p, rv, wts, split, mt, b, kvh, tid); break;
+                case 4: merge_rows<D, 4>(p, rv, wts, split, mt, b, kvh, tid); break;
+                case 5: merge_rows<D, 5>(p, rv, wts, split, mt, b, kvh, tid); break;
+                case 6: merge_rows<D, 6>(p, rv, wts, split, mt, b, kvh, tid); break;
+                case 7: merge_rows<D, 7>(p, rv, wts, split, mt, b, kvh, tid); break;
+                default: merge_rows<D, 8>(p, rv, wts, split, mt, b, kvh, tid); break;
+            }
+        }
+    }
+    // second phase of the cluster barrier: every CTA has received all its blocks, so no copy is in flight into
+    // or out of any CTA of the cluster when it exits
+    tc::cluster_arrive_relaxed();
+    tc::cluster_wait();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tbase, 512);
     }
     if (tid == 0 && *abort_flag) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
 }
@@ -777,10 +830,10 @@ template <int D>
 cudaError_t launch(const AttnParams &p, cudaStream_t s) {
     CUtensorMap kc, vc, kn, vn, qm;
     const cuuint64_t cache_rows =
-        p.block_table ? (cuuint64_t)p.num_pages * p.Hkv * TN : (cuuint64_t)p.B * p.Hkv * p.P_max;
+        p.block_table ? (cuuint64_t)p.num_pages * p.Hkv * kPageRows : (cuuint64_t)p.B * p.Hkv * p.P_max;
     const cuuint64_t dc[2] = {(cuuint64_t)D, cache_rows};
     const cuuint64_t sc[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t bc[2] = {64, TN};
+    const cuuint32_t bc[2] = {64, (cuuint32_t)(p.block_table ? BOXR : TN)};
     const cuuint64_t dn[3] = {(cuuint64_t)D, (cuuint64_t)p.Hkv, (cuuint64_t)p.B * p.R};
     const cuuint64_t sn[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.Hkv * D * 2};
     const cuuint32_t bn[3] = {64, 1, TN};
