@@ -8,10 +8,10 @@
 //
 // Warp roles (12 warps):
 //   warps 0, 2  TMA producers of K and of V (128-byte swizzle), each into its
-//               own 3-stage ring: prefix tiles from the cache (two 64-row
-//               boxes per tile: with a paged cache each box is one page), new-
-//               key tiles from K_new/V_new through a 3-D tensor map (no head
-//               gather).  A K stage is freed when its QK^T completes, a V
+//               own 3-stage ring: prefix tiles from the cache (one 128-row
+//               box per 64 columns; with a paged cache one 64-row box per
+//               page, two per tile), new-key tiles from K_new/V_new through a
+//               3-D tensor map (no head gather).  A K stage is freed when its QK^T completes, a V
 //               stage when its PV does, so K runs ahead of V.
 //   warp 1      TMEM owner; one thread issues S = Q K^T (tcgen05.mma, both
 //               operands in shared memory) into S buffer j % 3.
@@ -46,9 +46,10 @@
 // before sending), and every CTA has received its blocks (before exit).
 //
 // Before the previous kernel in the stream has finished (programmatic
-// dependent launch), a CTA sets up its barriers and TMEM and asks L2 for the
-// first K/V tiles of its run, from a prefix length read as a hint; the real
-// copies, and every read the results depend on, wait for that kernel.
+// dependent launch), a CTA sets up its barriers, tensor maps and TMEM; every
+// global read (prefix lengths, Q, K/V) waits for that kernel.  The first
+// tiles are then requested K, V, K, V, ... so the first PV's operand is not
+// queued behind every K stage.
 //
 // Every wait is bounded (p.wait_cycles).  On expiry the CTA raises
 // TIDAR_DEV_TIMEOUT in dev_status and every role stops; then the producers
@@ -347,29 +348,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::tma_prefetch_desc(&tm_vc);
         tc::tma_prefetch_desc(&tm_kn);
         tc::tma_prefetch_desc(&tm_vn);
-        // L2 hint for the first cache tiles of this CTA's run, from the prefix length as it reads now (the
-        // previous kernel may still change it: a wrong guess only costs traffic, L2 stays coherent)
-        const int P_hint = __ldcg(p.prefix_len + b);
-        if (P_hint >= 0 && P_hint <= p.P_max) {
-            int TPh, h0, h1;
-            split_range(P_hint, p.R, split, S, TPh, h0, h1);
-            for (int t = h0; t < min(h1, min(h0 + STAGES, TPh)); ++t) {
-                for (int h2 = 0; h2 < (p.block_table ? 2 : 1); ++h2) {
-                    int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
-                    if (p.block_table) {
-                        if (2 * t + h2 >= p.max_pages) continue;
-                        const int pg = __ldcg(p.block_table + (size_t)b * p.max_pages + 2 * t + h2);
-                        if (pg < 0 || pg >= p.num_pages) continue;
-                        y = (pg * p.Hkv + kvh) * BOXR;
-                    }
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) {
-                        tc::tma_prefetch_l2_2d(&tm_kc, h * 64, y);
-                        tc::tma_prefetch_l2_2d(&tm_vc, h * 64, y);
-                    }
-                }
-            }
-        }
     }
     if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
     // every global read below (prefix lengths, Q, K/V) waits for the previous kernel
@@ -454,8 +432,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---- thread 0 starts the first copies at once ----
     const int prologue = min(n, STAGES);
     if (tid == 0) {
-        for (int i = 0; i < prologue; ++i) issue_tile(i, 0);
-        for (int i = 0; i < prologue; ++i) issue_tile(i, 1);
+        for (int i = 0; i < prologue; ++i) {
+            issue_tile(i, 0);
+            issue_tile(i, 1);
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
