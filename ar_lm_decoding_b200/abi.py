@@ -42,6 +42,9 @@ _SIGS = {
     "tidar_attn_step_paged": (_i, [_vp] * 6 + [_i, _i, _vp] + [_i] * 5 + [_f, _i] + [_vp, _vp, _vp, _vp]),
     "tidar_kv_commit_paged": (_i, [_vp] * 5 + [_i] * 7 + [_vp] * 4 + [_i, _i, _vp] + [_vp] * 4 + [_sz, _vp, _vp]),
     "tidar_rope_qkv": (_i, [_vp, _vp] + [_i] * 5 + [ctypes.c_double] + [_vp] * 5),
+    "tidar_verify_commit_workspace_size": (_sz, [_i] * 3),
+    "tidar_verify_commit": (_i, [_vp, _vp, _i] + [_vp] * 4 + [_f] + [_vp] * 5 + [_i] * 9 + [_vp] * 12
+                            + [_vp, _sz, _vp, _vp]),
     "tidar_testing_attn_step_stalled": (_i, [_vp] * 6 + [_i] * 6 + [_f, _i] + [_vp, _vp, _vp, ctypes.c_longlong, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -168,6 +171,26 @@ def tidar_kv_commit(k_caches, v_caches, k_news, v_news, L, B, Hkv, D, k, P_max, 
         _ptr(k_caches), _ptr(v_caches), _ptr(k_news), _ptr(v_news), L, B, Hkv, D, k, P_max, _ptr(prefix_len),
         _ptr(accept_len), _ptr(resampled), _ptr(group_logits), logits_dtype, V, _ptr(u_draft), _ptr(next_drafts),
         _ptr(next_preaccepted), _ptr(next_q_group), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+
+
+def tidar_verify_commit_workspace_size(B, k, V) -> int:
+    return _lib.tidar_verify_commit_workspace_size(B, k, V)
+
+
+def tidar_verify_commit(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u_res, trust_ar, k_caches,
+                        v_caches, k_news, v_news, block_table, max_pages, num_pages, L, B, Hkv, D, k, P_max, V,
+                        prefix_len, group_logits, u_draft, accept_len, resampled, tokens, n_emitted, logp_d, logq_d,
+                        next_drafts, next_preaccepted, next_q_group, workspace, ws_bytes, dev_status,
+                        stream=None) -> None:
+    """tidar_verify_trust_mix followed by tidar_kv_commit (or its paged form when block_table is given) in one
+    launch."""
+    _check("tidar_verify_commit", _lib.tidar_verify_commit(
+        _ptr(p_logits), _ptr(q_logits), logits_dtype, _ptr(drafts), _ptr(preaccepted), _ptr(u_acc), _ptr(u_res),
+        trust_ar, _ptr(k_caches), _ptr(v_caches), _ptr(k_news), _ptr(v_news), _ptr(block_table), max_pages,
+        num_pages, L, B, Hkv, D, k, P_max, V, _ptr(prefix_len), _ptr(group_logits), _ptr(u_draft),
+        _ptr(accept_len), _ptr(resampled), _ptr(tokens), _ptr(n_emitted), _ptr(logp_d), _ptr(logq_d),
+        _ptr(next_drafts), _ptr(next_preaccepted), _ptr(next_q_group), _ptr(workspace), ws_bytes,
+        _ptr(dev_status), _stream(stream)))
 
 
 def tidar_expected_tokens_per_step(k, alpha) -> float:

@@ -14,6 +14,12 @@ size_t commit_workspace_bytes(int B, int k, int V);
 cudaError_t commit_launch(void *const *, void *const *, const void *const *, const void *const *, int, int, int, int,
                           int, int, int32_t *, const int32_t *, const int32_t *, const void *, int, int, const float *,
                           int32_t *, uint8_t *, int32_t *, void *, int32_t *, cudaStream_t, const int32_t *, int, int);
+size_t verify_commit_workspace_bytes(int B, int k, int V);
+cudaError_t verify_commit_launch(const void *, const void *, int, const int32_t *, const uint8_t *, const float *,
+                                 const float *, float, void *const *, void *const *, const void *const *,
+                                 const void *const *, const int32_t *, int, int, int, int, int, int, int, int, int,
+                                 int32_t *, const void *, const float *, int32_t *, int32_t *, int32_t *, int32_t *,
+                                 float *, float *, int32_t *, uint8_t *, int32_t *, void *, int32_t *, cudaStream_t);
 
 namespace {
 
@@ -152,7 +158,7 @@ tidar_status tidar_testing_attn_step_stalled(const void *q, const void *k_new, c
 }
 
 size_t tidar_verify_workspace_size(int B, int k, int V) {
-    if (B < 1 || k < 1 || k > kMaxDraft || V < 1) return 0;
+    if (B < 1 || k < 1 || k > kMaxDraft || V < 1 || V > kMaxVocab) return 0;
     return verify_workspace_bytes(B, k, V);
 }
 
@@ -164,7 +170,7 @@ tidar_status tidar_verify_trust_mix(const void *p_logits, const void *q_logits, 
                                     void *stream) {
     if (B < 1 || k < 1 || V < 1) return TIDAR_ERR_INVALID_ARG;
     if (!(trust_ar >= 0.f && trust_ar <= 1.f)) return TIDAR_ERR_INVALID_ARG;
-    if (k > kMaxDraft) return TIDAR_ERR_UNSUPPORTED;
+    if (k > kMaxDraft || V > kMaxVocab) return TIDAR_ERR_UNSUPPORTED;
     if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
     if (!p_logits || !q_logits || !drafts || !preaccepted || !u_acc || !u_res || !accept_len || !resampled ||
         !tokens || !n_emitted || !workspace || !dev_status)
@@ -187,7 +193,7 @@ tidar_status tidar_verify(const void *p_logits, const void *q_logits, int logits
 }
 
 size_t tidar_kv_commit_workspace_size(int B, int k, int V) {
-    if (B < 1 || k < 1 || k > kMaxDraft || V < 1) return 0;
+    if (B < 1 || k < 1 || k > kMaxDraft || V < 1 || V > kMaxVocab) return 0;
     return commit_workspace_bytes(B, k, V);
 }
 
@@ -198,7 +204,7 @@ tidar_status tidar_kv_commit(void *const *k_caches, void *const *v_caches, const
                              int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group, void *workspace,
                              size_t ws_bytes, int32_t *dev_status, void *stream) {
     if (L < 1 || B < 1 || Hkv < 1 || k < 1 || V < 1 || P_max < 0) return TIDAR_ERR_INVALID_ARG;
-    if (k > kMaxDraft || (D != 64 && D != 128)) return TIDAR_ERR_UNSUPPORTED;
+    if (k > kMaxDraft || V > kMaxVocab || (D != 64 && D != 128)) return TIDAR_ERR_UNSUPPORTED;
     if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
     if (!k_caches || !v_caches || !k_news || !v_news || !prefix_len || !accept_len || !resampled || !group_logits ||
         !u_draft || !next_drafts || !next_preaccepted || !next_q_group || !workspace || !dev_status)
@@ -221,7 +227,7 @@ tidar_status tidar_kv_commit_paged(void *const *k_pools, void *const *v_pools, c
     if (!block_table || max_pages < 1 || num_pages < 1) return TIDAR_ERR_INVALID_ARG;
     if (max_pages > kMaxPagesPerSeq) return TIDAR_ERR_UNSUPPORTED;
     if (L < 1 || B < 1 || Hkv < 1 || k < 1 || V < 1) return TIDAR_ERR_INVALID_ARG;
-    if (k > kMaxDraft || (D != 64 && D != 128)) return TIDAR_ERR_UNSUPPORTED;
+    if (k > kMaxDraft || V > kMaxVocab || (D != 64 && D != 128)) return TIDAR_ERR_UNSUPPORTED;
     if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
     if (!k_pools || !v_pools || !k_news || !v_news || !prefix_len || !accept_len || !resampled || !group_logits ||
         !u_draft || !next_drafts || !next_preaccepted || !next_q_group || !workspace || !dev_status)
@@ -232,6 +238,46 @@ tidar_status tidar_kv_commit_paged(void *const *k_pools, void *const *v_pools, c
                                   accept_len, resampled, group_logits, logits_dtype, V, u_draft, next_drafts,
                                   next_preaccepted, next_q_group, workspace, dev_status,
                                   static_cast<cudaStream_t>(stream), block_table, max_pages, num_pages));
+}
+
+size_t tidar_verify_commit_workspace_size(int B, int k, int V) {
+    if (B < 1 || k < 1 || k > kMaxDraft || V < 1 || V > kMaxVocab) return 0;
+    return verify_commit_workspace_bytes(B, k, V);
+}
+
+tidar_status tidar_verify_commit(const void *p_logits, const void *q_logits, int logits_dtype, const int32_t *drafts,
+                                 const uint8_t *preaccepted, const float *u_acc, const float *u_res, float trust_ar,
+                                 void *const *k_caches, void *const *v_caches, const void *const *k_news,
+                                 const void *const *v_news, const int32_t *block_table, int max_pages, int num_pages,
+                                 int L, int B, int Hkv, int D, int k, int P_max, int V, int32_t *prefix_len,
+                                 const void *group_logits, const float *u_draft, int32_t *accept_len,
+                                 int32_t *resampled, int32_t *tokens, int32_t *n_emitted, float *logp_d,
+                                 float *logq_d, int32_t *next_drafts, uint8_t *next_preaccepted,
+                                 int32_t *next_q_group, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 void *stream) {
+    if (L < 1 || B < 1 || Hkv < 1 || k < 1 || V < 1) return TIDAR_ERR_INVALID_ARG;
+    if (!(trust_ar >= 0.f && trust_ar <= 1.f)) return TIDAR_ERR_INVALID_ARG;
+    if (k > kMaxDraft || V > kMaxVocab || (D != 64 && D != 128)) return TIDAR_ERR_UNSUPPORTED;
+    if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
+    if (block_table) {
+        if (max_pages < 1 || num_pages < 1) return TIDAR_ERR_INVALID_ARG;
+        if (max_pages > kMaxPagesPerSeq) return TIDAR_ERR_UNSUPPORTED;
+        P_max = max_pages * kPageRows;
+    } else if (P_max < 0) {
+        return TIDAR_ERR_INVALID_ARG;
+    }
+    if (!p_logits || !q_logits || !drafts || !preaccepted || !u_acc || !u_res || !k_caches || !v_caches ||
+        !k_news || !v_news || !prefix_len || !group_logits || !u_draft || !accept_len || !resampled || !tokens ||
+        !n_emitted || !next_drafts || !next_preaccepted || !next_q_group || !workspace || !dev_status)
+        return TIDAR_ERR_INVALID_ARG;
+    if (!aligned256(workspace)) return TIDAR_ERR_INVALID_ARG;
+    if (ws_bytes < verify_commit_workspace_bytes(B, k, V)) return TIDAR_ERR_WORKSPACE;
+    return launched(verify_commit_launch(p_logits, q_logits, logits_dtype, drafts, preaccepted, u_acc, u_res,
+                                         trust_ar, k_caches, v_caches, k_news, v_news, block_table,
+                                         block_table ? max_pages : 0, block_table ? num_pages : 0, L, B, Hkv, D, k,
+                                         P_max, V, prefix_len, group_logits, u_draft, accept_len, resampled, tokens,
+                                         n_emitted, logp_d, logq_d, next_drafts, next_preaccepted, next_q_group,
+                                         workspace, dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 const char *tidar_status_string(tidar_status s) {

@@ -18,6 +18,7 @@ constexpr int kNumSMs = 148;
 constexpr int kMaxDraft = 16;  // longest draft block k every entry point accepts
 constexpr int kPageRows = 64;  // rows of a KV-cache page: one key tile of the attention kernel
 constexpr int kMaxPagesPerSeq = 1024;  // longest block-table row a paged call accepts (65536 cached tokens)
+constexpr int kMaxVocab = 1 << 19;      // largest vocabulary the verify and commit accept (64 chunks of 8192)
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }

@@ -65,7 +65,7 @@ tidar_status tidar_verify_noalloc(const void *p_logits, const void *q_logits, in
                                   int32_t *tokens, int32_t *n_emitted, float *logp_d, float *logq_d,
                                   int32_t *dev_status, void *stream) {
     if (B < 1 || k < 1 || V < 1) return TIDAR_ERR_INVALID_ARG;
-    if (k > tidar::kMaxDraft) return TIDAR_ERR_UNSUPPORTED;
+    if (k > tidar::kMaxDraft || V > tidar::kMaxVocab) return TIDAR_ERR_UNSUPPORTED;
     if (logits_dtype != TIDAR_DT_BF16 && logits_dtype != TIDAR_DT_F32) return TIDAR_ERR_INVALID_ARG;
     if (!p_logits || !q_logits || !drafts || !preaccepted || !u_acc || !u_res || !accept_len || !resampled ||
         !tokens || !n_emitted || !dev_status)

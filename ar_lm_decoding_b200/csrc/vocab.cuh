@@ -9,6 +9,7 @@ namespace tidar {
 
 constexpr int kChunk = 8192;        // vocabulary entries per CTA
 constexpr int kStatThreads = 256;   // kChunk / kStatThreads = 32 entries per thread
+static_assert(kMaxVocab == 64 * kChunk, "a row's chunk statistics are held two per lane of one warp");
 
 struct ChunkStat {
     float m;   // max logit of the chunk

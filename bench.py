@@ -1,4 +1,5 @@
-"""Benchmark of one TiDAR decode step on B200: L x tidar_attn_step + tidar_verify + tidar_kv_commit.
+"""Benchmark of one TiDAR decode step on B200: L x tidar_attn_step + tidar_verify_commit (the verify and the
+commit in one launch).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
@@ -249,7 +250,9 @@ class Step:
         self.ws_attn_n = abi.tidar_attn_workspace_size(B, Hq, Hkv, D, k, Pm)
         self.ws_ver_n = abi.tidar_verify_workspace_size(B, k, V)
         self.ws_com_n = abi.tidar_kv_commit_workspace_size(B, k, V)
-        self.ws = torch.empty(max(self.ws_attn_n, self.ws_ver_n, self.ws_com_n), dtype=torch.uint8, device=device)
+        self.ws_vc_n = abi.tidar_verify_commit_workspace_size(B, k, V)
+        self.ws = torch.empty(max(self.ws_attn_n, self.ws_ver_n, self.ws_com_n, self.ws_vc_n), dtype=torch.uint8,
+                              device=device)
         self.scale = 1.0 / math.sqrt(D)
         self.launches_per_step = None
 
@@ -272,13 +275,21 @@ class Step:
                                  self.u_draft, self.next_drafts, self.next_pre, self.next_q_group, self.ws,
                                  self.ws.numel(), self.status, stream)
 
+    def verify_commit(self, stream):
+        c = self.cfg
+        self.abi.tidar_verify_commit(self.p_logits, self.q_logits, self.ldt, self.drafts, self.pre_u8, self.u_acc,
+                                     self.u_res, 1.0, self.kc_ptrs, self.vc_ptrs, self.kn_ptrs, self.vn_ptrs, None, 0,
+                                     0, c.L, c.B, c.Hkv, c.D, c.k, c.P_max, c.V, self.prefix, self.g_logits,
+                                     self.u_draft, self.accept_len, self.resampled, self.tokens, self.n_emitted,
+                                     self.logp, self.logq, self.next_drafts, self.next_pre, self.next_q_group,
+                                     self.ws, self.ws.numel(), self.status, stream)
+
     def run(self, stream):
         """One decode step (prefix length restored first so every step sees the same prefix)."""
         self.prefix.copy_(self.prefix0)
         for l in range(self.cfg.L):
             self.attn(l, stream)
-        self.verify(stream)
-        self.commit(stream)
+        self.verify_commit(stream)
 
 
 def gpu_smi_id(device):
@@ -320,9 +331,9 @@ def job_throughput(world, step_s):
 
 
 def kernels_per_step(cfg):
-    # per layer: one attention kernel (split-KV merged in-kernel); verify: one cooperative kernel; commit: one
-    # cooperative kernel (their grid-barrier counters are zeroed by memset nodes, not kernels)
-    return cfg.L + 2
+    # per layer: one attention kernel (split-KV merged in-kernel); verify + commit: one cooperative kernel (its
+    # counters are zeroed by a memset node, not a kernel)
+    return cfg.L + 1
 
 
 def init_ranks(backend):
@@ -434,10 +445,15 @@ def gpu_arm(args, cfg):
     torch.cuda.synchronize()
     attn_ms_launch = max_over_ranks(a0.elapsed_time(a1) / (reps * cfg.L))
     del attn_graph
+    # the step's verify + commit launch, and (for comparison) the two separate calls it replaces; each graph
+    # restores the prefix length first (a 4-byte copy node)
     breakdown = {"attn_us_per_launch": round(attn_ms_launch * 1e3, 3),
-                 "verify_us": round(graph_us(stream, reps, lambda: step.verify(stream.cuda_stream)), 3),
-                 "commit_us": round(graph_us(stream, reps, lambda: (step.prefix.copy_(step.prefix0),
-                                                                    step.commit(stream.cuda_stream))), 3)}
+                 "verify_commit_us": round(graph_us(stream, reps, lambda: (step.prefix.copy_(step.prefix0),
+                                                                           step.verify_commit(stream.cuda_stream))),
+                                           3),
+                 "separate_verify_us": round(graph_us(stream, reps, lambda: step.verify(stream.cuda_stream)), 3),
+                 "separate_commit_us": round(graph_us(stream, reps, lambda: (step.prefix.copy_(step.prefix0),
+                                                                             step.commit(stream.cuda_stream))), 3)}
 
     e2e = e2e_leg(step, stream, args, barrier, max_over_ranks, world)
 
@@ -522,7 +538,7 @@ def graph_us(stream, reps, fn):
 
 def e2e_step(step, stream, copy_stream, events, pin_in, pin_out):
     """One decode step through the C ABI as a user runs it: this step's inputs (every layer's Q / K_new /
-    V_new, the p / q / group logits, drafts and uniforms) copied from pinned host memory, the L + 2 library
+    V_new, the p / q / group logits, drafts and uniforms) copied from pinned host memory, the L + 1 library
     calls, the results copied back and read on the host.  The input copies are issued layer by layer on a
     second stream, so that layer l's inputs cross the host link while layer l-1 computes; every attention call
     waits only for its own layer's inputs."""
@@ -539,8 +555,7 @@ def e2e_step(step, stream, copy_stream, events, pin_in, pin_out):
             stream.wait_event(events[l])
             step.attn(l, stream.cuda_stream)
         stream.wait_event(events[-1])
-        step.verify(stream.cuda_stream)
-        step.commit(stream.cuda_stream)
+        step.verify_commit(stream.cuda_stream)
         pin_out.copy_(step.outbuf[:step.out_bytes], non_blocking=True)
     stream.synchronize()
     return int(pin_out[:4].view(torch.int32).item())  # the accept length of sequence 0, read on the host

@@ -12,7 +12,8 @@
  * Three calls cover that hot path:
  *   tidar_attn_step   the structured hybrid-mask attention of one layer;
  *   tidar_verify      the AR rejection-sampling verify of the drafts;
- *   tidar_kv_commit   the exact-KV-cache commit/evict + next-draft selection.
+ *   tidar_kv_commit   the exact-KV-cache commit/evict + next-draft selection;
+ * tidar_verify_commit makes the last two in one launch.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -191,6 +192,7 @@ size_t tidar_verify_workspace_size(int B, int k, int V);
  * n_emitted  int32 [B]
  * logp_d, logq_d  f32 [B, k] or NULL: log p_i(d_i), log q_i(d_i)
  * dev_status TIDAR_DEV_BAD_TOKEN when a draft is outside [0, V).
+ * V <= 524288 (else TIDAR_ERR_UNSUPPORTED).
  */
 tidar_status tidar_verify(const void *p_logits, const void *q_logits, int logits_dtype,
                           const int32_t *drafts, const uint8_t *preaccepted,
@@ -283,6 +285,7 @@ size_t tidar_kv_commit_workspace_size(int B, int k, int V);
  * dev_status  TIDAR_DEV_BAD_ACCEPT / TIDAR_DEV_BAD_PREFIX / TIDAR_DEV_BAD_TOKEN
  *             when accept_len, P_b + j* or resampled is out of range; that
  *             sequence is then left untouched.
+ * V <= 524288 (else TIDAR_ERR_UNSUPPORTED).
  */
 tidar_status tidar_kv_commit(void *const *k_caches, void *const *v_caches,
                              const void *const *k_news, const void *const *v_news,
@@ -343,6 +346,52 @@ tidar_status tidar_kv_commit_paged(void *const *k_pools, void *const *v_pools,
                                    const void *group_logits, int logits_dtype, int V, const float *u_draft,
                                    int32_t *next_drafts, uint8_t *next_preaccepted, int32_t *next_q_group,
                                    void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Verify + commit in one launch                                             */
+/* ------------------------------------------------------------------------ */
+
+size_t tidar_verify_commit_workspace_size(int B, int k, int V);
+
+/*
+ * tidar_verify_trust_mix followed by tidar_kv_commit (tidar_kv_commit_paged
+ * when block_table is not NULL) as one launch: the verify's accept length j*
+ * and replacement token feed the commit directly.
+ *
+ * Defined by: the same passages as the two calls it replaces (TiDAR summary
+ * §3.2 "Talk" / "Think": the drafts are verified, the KV of the accepted ones
+ * is kept, and the pre-drafts of the group matching the accept outcome become
+ * the next drafts -- all within one decode step).  The results are those of
+ * the two calls made in turn on the same arguments, with these differences:
+ *  - the commit's P_b is prefix_len[b] as it was when the call started (the
+ *    commit never reads its own update);
+ *  - a sequence with a draft outside [0, V) (TIDAR_DEV_BAD_TOKEN) is left
+ *    untouched by the commit, since it has no accept length;
+ *  - with a block table, P_max is ignored (the capacity is max_pages * 64);
+ *    block_table, max_pages and num_pages are as for tidar_kv_commit_paged;
+ *  - if the replacement draw finds no token (every weight zero, which only an
+ *    all -inf row allows), TIDAR_DEV_BAD_TOKEN is set and the sequence's
+ *    state (prefix_len, next_q_group, next_preaccepted, next_drafts[b][0]) is
+ *    not advanced; cache rows P_b .. P_b + j* - 1 may have been written.
+ * The verify outputs (accept_len, resampled, tokens, n_emitted, logp_d,
+ * logq_d) are written as tidar_verify writes them, also for a sequence whose
+ * commit inputs are invalid (prefix or page; that sequence's commit is
+ * skipped with the matching TIDAR_DEV_* bit).  trust_ar = 1 is the plain AR
+ * verify.  V <= 524288.  The workspace is tidar_verify_commit_workspace_size
+ * bytes, 256-byte aligned.
+ */
+tidar_status tidar_verify_commit(const void *p_logits, const void *q_logits, int logits_dtype,
+                                 const int32_t *drafts, const uint8_t *preaccepted,
+                                 const float *u_acc, const float *u_res, float trust_ar,
+                                 void *const *k_caches, void *const *v_caches,
+                                 const void *const *k_news, const void *const *v_news,
+                                 const int32_t *block_table, int max_pages, int num_pages,
+                                 int L, int B, int Hkv, int D, int k, int P_max, int V,
+                                 int32_t *prefix_len, const void *group_logits, const float *u_draft,
+                                 int32_t *accept_len, int32_t *resampled, int32_t *tokens, int32_t *n_emitted,
+                                 float *logp_d, float *logq_d, int32_t *next_drafts, uint8_t *next_preaccepted,
+                                 int32_t *next_q_group, void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *tidar_status_string(tidar_status s);

@@ -31,7 +31,7 @@ def test_algorithmic_bytes_closed_form():
 
 def test_kernels_per_step():
     cfg = synth.CONFIGS["qwen3-8b_k8"]
-    assert bench.kernels_per_step(cfg) == cfg.L + 2  # L attention launches, verify (1), commit (1)
+    assert bench.kernels_per_step(cfg) == cfg.L + 1  # L attention launches, verify + commit (1)
 
 
 def test_clock_sample_parsing():

@@ -4,7 +4,8 @@ One step is the pages' decode step ("TiDAR: Think in Diffusion, Talk in Autoregr
 summary, "并行 self-speculative 生成 (§3.2)"; notes.yuuk.io talk notes, §推論パイプライン): the forward over
 [cached prefix | k drafts | k+1 pre-draft groups] (here: L tidar_attn_step calls), the AR rejection-sampling
 verify of the drafts (tidar_verify), then the exact-KV commit and the choice of the next draft block from group
-j* (tidar_kv_commit).  The state a step hands to the next stays where a caller keeps it:
+j* (tidar_kv_commit) -- or those two as one tidar_verify_commit call.  The state a step hands to the next stays
+where a caller keeps it:
 
 * on the GPU side, on the device: the per-layer KV caches and prefix_len (updated in place by the commit and
   read by the next step's attention), next_drafts and next_preaccepted (the next step's drafts and pre-accepted
@@ -97,8 +98,10 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["verify+commit", "verify_commit"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_decode_loop_matches_oracle(name):
+def test_decode_loop_matches_oracle(name, fused):
+    """fused: the verify and the commit as one tidar_verify_commit call."""
     steps = 5
     cfg0 = CASES[name]
     # capacity for every step accepting the whole block
@@ -126,8 +129,8 @@ def test_decode_loop_matches_oracle(name):
     g_q = _logits_dev(vin["q_logits"])
     dt = abi.TIDAR_DT_BF16 if cfg.logits_dtype == "bf16" else abi.TIDAR_DT_F32
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    ws = torch.empty(max(abi.tidar_verify_workspace_size(B, k, V), abi.tidar_kv_commit_workspace_size(B, k, V)),
-                     dtype=torch.uint8, device=DEV)
+    ws = torch.empty(max(abi.tidar_verify_workspace_size(B, k, V), abi.tidar_kv_commit_workspace_size(B, k, V),
+                         abi.tidar_verify_commit_workspace_size(B, k, V)), dtype=torch.uint8, device=DEV)
     report, accept_seen = [], []
     for step in range(steps):
         # fresh model outputs of this step
@@ -156,14 +159,24 @@ def test_decode_loop_matches_oracle(name):
         nem = torch.full((B,), -7, dtype=torch.int32, device=DEV)
         lp = torch.zeros((B, k), dtype=torch.float32, device=DEV)
         lq = torch.zeros((B, k), dtype=torch.float32, device=DEV)
-        abi.tidar_verify(g_p, g_q, dt, g_drafts, g_pre, torch.from_numpy(u_acc).to(DEV),
-                         torch.from_numpy(u_res).to(DEV), B, k, V, acc, res, tok, nem, lp, lq, ws, ws.numel(), status)
         nd = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
         npre = torch.full((B,), 7, dtype=torch.uint8, device=DEV)
         nqg = torch.full((B,), -7, dtype=torch.int32, device=DEV)
-        abi.tidar_kv_commit(abi.pointer_array(g_kc, DEV), abi.pointer_array(g_vc, DEV), abi.pointer_array(g_kn, DEV),
-                            abi.pointer_array(g_vn, DEV), L, B, Hkv, D, k, P_max, g_pl, acc, res, g_g, dt, V,
-                            torch.from_numpy(u_draft).to(DEV), nd, npre, nqg, ws, ws.numel(), status)
+        if fused:
+            abi.tidar_verify_commit(g_p, g_q, dt, g_drafts, g_pre, torch.from_numpy(u_acc).to(DEV),
+                                    torch.from_numpy(u_res).to(DEV), 1.0, abi.pointer_array(g_kc, DEV),
+                                    abi.pointer_array(g_vc, DEV), abi.pointer_array(g_kn, DEV),
+                                    abi.pointer_array(g_vn, DEV), None, 0, 0, L, B, Hkv, D, k, P_max, V, g_pl, g_g,
+                                    torch.from_numpy(u_draft).to(DEV), acc, res, tok, nem, lp, lq, nd, npre, nqg, ws,
+                                    ws.numel(), status)
+        else:
+            abi.tidar_verify(g_p, g_q, dt, g_drafts, g_pre, torch.from_numpy(u_acc).to(DEV),
+                             torch.from_numpy(u_res).to(DEV), B, k, V, acc, res, tok, nem, lp, lq, ws, ws.numel(),
+                             status)
+            abi.tidar_kv_commit(abi.pointer_array(g_kc, DEV), abi.pointer_array(g_vc, DEV),
+                                abi.pointer_array(g_kn, DEV), abi.pointer_array(g_vn, DEV), L, B, Hkv, D, k, P_max,
+                                g_pl, acc, res, g_g, dt, V, torch.from_numpy(u_draft).to(DEV), nd, npre, nqg, ws,
+                                ws.numel(), status)
         torch.cuda.synchronize()
         assert status.item() == 0, (step, status.item())
 

@@ -1,4 +1,4 @@
-"""Paged KV cache (tidar_attn_step_paged, tidar_kv_commit_paged) on the GPU.
+"""Paged KV cache (tidar_attn_step_paged, tidar_kv_commit_paged, tidar_verify_commit with a block table) on the GPU.
 
 A paged cache is a storage layout: cache row n of sequence b is row n % 64 of page block_table[b][n / 64] of a
 pool shared by all sequences.  The tests scatter the rows of contiguous caches over randomly permuted pages of a
@@ -134,7 +134,8 @@ def test_paged_attention_bad_page_sets_status_and_skips():
     assert np.abs(o[0] - o_ref[0]).max() <= O_TOL and np.abs(lse[0] - lse_ref[0]).max() <= LSE_TOL
 
 
-def test_paged_continuous_batching_loop():
+@pytest.mark.parametrize("fused", [False, True], ids=["verify+commit", "verify_commit"])
+def test_paged_continuous_batching_loop(fused):
     """Four sequence slots decode for six steps; when a slot's sequence reaches its length it is replaced by a
     new sequence (fresh prefix in fresh pages).  Attention (2 layers), verify and the paged commit run on the
     GPU with the block table and pools on the device; the oracle runs the same steps on gathered contiguous
@@ -165,8 +166,8 @@ def test_paged_continuous_batching_loop():
     vin = synth.make_verify_inputs(cfg.with_(peaks=True), seed=4)
     drafts, q_log, pre = vin["drafts"].copy(), vin["q_logits"].copy(), vin["preaccepted"].copy()
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    ws = torch.empty(max(abi.tidar_verify_workspace_size(B, k, V), abi.tidar_kv_commit_workspace_size(B, k, V)),
-                     dtype=torch.uint8, device=DEV)
+    ws = torch.empty(max(abi.tidar_verify_workspace_size(B, k, V), abi.tidar_kv_commit_workspace_size(B, k, V),
+                         abi.tidar_verify_commit_workspace_size(B, k, V)), dtype=torch.uint8, device=DEV)
     report, turnovers = [], 0
     for step in range(6):
         table_d = torch.from_numpy(pool.table).to(DEV)
@@ -196,22 +197,42 @@ def test_paged_continuous_batching_loop():
         v_inp = dict(p_logits=synth.f32_to_bf16_bits(zp), q_logits=q_log, drafts=drafts, preaccepted=pre,
                      u_acc=rng.random((B, k)).astype(np.float32), u_res=rng.random(B).astype(np.float32))
         import tidar_gpu
-        got_v = tidar_gpu.verify(v_inp)
-        ref_v = compare_verify(v_inp, got_v, report)
-        # paged commit on the GPU
         u_draft = rng.random((B, k)).astype(np.float32)
         g_kn = [_bf16_dev(kn[l]) for l in range(L)]
         g_vn = [_bf16_dev(vn[l]) for l in range(L)]
         nd = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
         npre = torch.full((B,), 7, dtype=torch.uint8, device=DEV)
         nqg = torch.full((B,), -7, dtype=torch.int32, device=DEV)
-        abi.tidar_kv_commit_paged(abi.pointer_array(g_kp, DEV), abi.pointer_array(g_vp, DEV),
-                                  abi.pointer_array(g_kn, DEV), abi.pointer_array(g_vn, DEV), table_d, max_pages,
-                                  num_pages, L, B, Hkv, D, k, g_pl,
-                                  torch.from_numpy(got_v["accept_len"]).to(DEV),
-                                  torch.from_numpy(got_v["resampled"]).to(DEV), _bf16_dev(g_logits),
-                                  abi.TIDAR_DT_BF16, V, torch.from_numpy(u_draft).to(DEV), nd, npre, nqg, ws,
-                                  ws.numel(), status)
+        if fused:  # verify and paged commit in one launch
+            outs = [torch.full((B,), -7, dtype=torch.int32, device=DEV) for _ in range(3)]
+            tok = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
+            lp = torch.zeros((B, k), dtype=torch.float32, device=DEV)
+            lq = torch.zeros((B, k), dtype=torch.float32, device=DEV)
+            abi.tidar_verify_commit(_bf16_dev(v_inp["p_logits"]), _bf16_dev(q_log), abi.TIDAR_DT_BF16,
+                                    torch.from_numpy(drafts.astype(np.int32)).to(DEV),
+                                    torch.from_numpy(pre.astype(np.uint8)).to(DEV),
+                                    torch.from_numpy(v_inp["u_acc"]).to(DEV), torch.from_numpy(v_inp["u_res"]).to(DEV),
+                                    1.0, abi.pointer_array(g_kp, DEV), abi.pointer_array(g_vp, DEV),
+                                    abi.pointer_array(g_kn, DEV), abi.pointer_array(g_vn, DEV), table_d, max_pages,
+                                    num_pages, L, B, Hkv, D, k, 0, V, g_pl, _bf16_dev(g_logits),
+                                    torch.from_numpy(u_draft).to(DEV), outs[0], outs[1], tok, outs[2], lp, lq, nd,
+                                    npre, nqg, ws, ws.numel(), status)
+            torch.cuda.synchronize()
+            got_v = dict(accept_len=outs[0].cpu().numpy(), resampled=outs[1].cpu().numpy(),
+                         tokens=tok.cpu().numpy(), n_emitted=outs[2].cpu().numpy(), logp_d=lp.cpu().numpy(),
+                         logq_d=lq.cpu().numpy())
+            ref_v = compare_verify(v_inp, got_v, report)
+        else:
+            got_v = tidar_gpu.verify(v_inp)
+            ref_v = compare_verify(v_inp, got_v, report)
+            # paged commit on the GPU
+            abi.tidar_kv_commit_paged(abi.pointer_array(g_kp, DEV), abi.pointer_array(g_vp, DEV),
+                                      abi.pointer_array(g_kn, DEV), abi.pointer_array(g_vn, DEV), table_d, max_pages,
+                                      num_pages, L, B, Hkv, D, k, g_pl,
+                                      torch.from_numpy(got_v["accept_len"]).to(DEV),
+                                      torch.from_numpy(got_v["resampled"]).to(DEV), _bf16_dev(g_logits),
+                                      abi.TIDAR_DT_BF16, V, torch.from_numpy(u_draft).to(DEV), nd, npre, nqg, ws,
+                                      ws.numel(), status)
         torch.cuda.synchronize()
         assert status.item() == 0
         c = oracle.kv_commit(o_kc, o_vc, kn, vn, prefix, ref_v["accept_len"], ref_v["resampled"], g_logits, u_draft)

@@ -1,4 +1,4 @@
-"""GPU parity of tidar_verify and tidar_kv_commit against the CPU oracle.
+"""GPU parity of tidar_verify, tidar_kv_commit and tidar_verify_commit against the CPU oracle.
 
 Accept lengths, emitted tokens, resampled tokens, next drafts and committed KV
 must be bit-exact given the same uniforms.  The only exemption: a decision
@@ -161,3 +161,83 @@ def test_step_chain_state_machine():
     for b in range(cfg.B):
         if got["accept_len"][b] < cfg.k:
             assert cg["next_drafts"][b, 0] == got["resampled"][b] and cg["next_preaccepted"][b] == 1
+
+
+def _check_fused(inp, got, kc, vc, kn, vn, pl, report, trust_ar=1.0):
+    """The fused call's outputs against the oracle's verify, then its commit on the verify's outcome."""
+    ref = compare_verify(inp, got, report, trust_ar=trust_ar)
+    c = oracle.kv_commit(kc, vc, kn, vn, pl, ref["accept_len"], ref["resampled"], inp["group_logits"], inp["u_draft"])
+    assert np.array_equal(got["k_caches"], c["k_caches"])
+    assert np.array_equal(got["v_caches"], c["v_caches"])
+    assert np.array_equal(got["prefix_len"], c["prefix_len"])
+    assert np.array_equal(got["next_q_group"], c["next_q_group"])
+    assert np.array_equal(got["next_preaccepted"], c["next_preaccepted"])
+    compare_next_drafts(got, c, inp["u_draft"], report)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen2.5-1.5b_k4", "qwen2.5-1.5b_k16", "qwen3-8b_k8", "qwen3-8b_k8_b8",
+                                  "qwen3-8b_k8_peaks", "qwen3-32b_k16"])
+def test_verify_commit_parity(name):
+    """One launch = tidar_verify then tidar_kv_commit: every output against the oracle's two steps."""
+    cfg = synth.CONFIGS[name]
+    report, seen = [], []
+    for seed in range(2):
+        inp = synth.make_verify_inputs(cfg, seed=seed)
+        kc, vc, kn, vn, pl, _, _, _, _ = _commit_inputs(cfg, seed, L=2)
+        got = _gpu().verify_commit(inp, kc, vc, kn, vn, pl)
+        _check_fused(inp, got, kc, vc, kn, vn, pl, report)
+        seen += got["accept_len"].tolist()
+    print(f"{name}: accept lengths {seen}, exemptions {report}")
+    assert len(report) <= 1
+
+
+@pytest.mark.parametrize("trust_ar", [0.0, 0.37])
+def test_verify_commit_trust_mix(trust_ar):
+    cfg = synth.CONFIGS["qwen2.5-1.5b_k4"].with_(B=4, V=30000, ragged=(100, 400))
+    report = []
+    for seed in range(2):
+        inp = synth.make_verify_inputs(cfg, seed=seed)
+        kc, vc, kn, vn, pl, _, _, _, _ = _commit_inputs(cfg, seed, L=2)
+        got = _gpu().verify_commit(inp, kc, vc, kn, vn, pl, trust_ar=trust_ar)
+        _check_fused(inp, got, kc, vc, kn, vn, pl, report, trust_ar=trust_ar)
+        if trust_ar == 0.0:
+            assert (got["accept_len"] == cfg.k).all()
+    assert len(report) <= 1
+
+
+def test_verify_commit_many_sequences():
+    """256 sequences on small vocabularies (several items per CTA in every phase), bf16 and f32."""
+    report = []
+    for V, k, dtype in ((8, 4, "f32"), (9000, 3, "bf16"), (17, 1, "bf16")):
+        cfg = synth.CONFIGS["tiny"].with_(B=256, V=V, k=k, logits_dtype=dtype, cfg_id=200 + V)
+        inp = synth.make_verify_inputs(cfg, seed=V)
+        kc, vc, kn, vn, pl, _, _, _, _ = _commit_inputs(cfg, V, L=1)
+        got = _gpu().verify_commit(inp, kc, vc, kn, vn, pl)
+        _check_fused(inp, got, kc, vc, kn, vn, pl, report)
+    assert len(report) <= 2
+
+
+def test_verify_commit_bad_inputs():
+    """A draft outside the vocabulary leaves its sequence untouched (no accept length); a prefix too close to
+    the capacity keeps the verify outputs but skips that sequence's commit; the others are committed."""
+    cfg = synth.CONFIGS["tiny"].with_(B=3)
+    inp = synth.make_verify_inputs(cfg, seed=11)
+    inp["drafts"] = inp["drafts"].copy()
+    inp["drafts"][1, 2] = cfg.V                             # b=1: a draft outside [0, V)
+    inp["preaccepted"] = np.zeros(3, inp["preaccepted"].dtype)
+    inp["u_acc"] = np.zeros_like(inp["u_acc"])              # every valid draft accepted: j* = k
+    kc, vc, kn, vn, _, _, _, _, _ = _commit_inputs(cfg, 11, L=2)
+    pl = np.array([cfg.P, cfg.P, cfg.P_max - 1], np.int32)  # b=2: P + j* beyond capacity
+    got = _gpu().verify_commit(inp, kc, vc, kn, vn, pl, want_status=True)
+    assert got["status"] & 2 and got["status"] & 1
+    assert list(got["prefix_len"]) == [cfg.P + cfg.k, cfg.P, cfg.P_max - 1]
+    assert np.array_equal(got["k_caches"][:, 1:], kc[:, 1:]) and np.array_equal(got["v_caches"][:, 1:], vc[:, 1:])
+    assert got["accept_len"][1] == -7 and got["next_q_group"][1] == -7 and got["next_q_group"][2] == -7
+    sub = {n: (v[[0, 2]] if hasattr(v, "shape") and v.shape[:1] == (3,) else v) for n, v in inp.items()}
+    ref = oracle.verify(sub)
+    assert list(got["accept_len"][[0, 2]]) == list(ref["accept_len"]) == [cfg.k, cfg.k]
+    assert np.array_equal(got["tokens"][[0, 2]], ref["tokens"])
+    c = oracle.kv_commit(kc[:, :1], vc[:, :1], kn[:, :1], vn[:, :1], pl[:1], ref["accept_len"][:1],
+                         ref["resampled"][:1], inp["group_logits"][:1], inp["u_draft"][:1])
+    assert np.array_equal(got["k_caches"][:, :1], c["k_caches"])
+    assert got["next_q_group"][0] == cfg.k and got["next_preaccepted"][0] == 0

@@ -116,3 +116,46 @@ def kv_commit(k_caches, v_caches, k_news, v_news, prefix_len, accept_len, resamp
     if not want_status:
         assert res["status"] == 0, f"device status {res['status']}"
     return res
+
+
+def verify_commit(inp: dict, k_caches, v_caches, k_news, v_news, prefix_len, trust_ar=1.0, want_status=False):
+    """tidar_verify_commit on the numpy verify inputs (with group_logits and u_draft) and contiguous caches
+    [L,B,Hkv,P_max,D] / new K/V [L,B,R,Hkv,D] (uint16 bf16 bits); returns host copies of every output."""
+    L, B, Hkv, P_max, D = k_caches.shape
+    p, dt = logits_dev(inp["p_logits"])
+    q, _ = logits_dev(inp["q_logits"])
+    g, _ = logits_dev(inp["group_logits"])
+    _, k, V = inp["p_logits"].shape
+    kc = [dev_u16_as_bf16(k_caches[l]) for l in range(L)]
+    vc = [dev_u16_as_bf16(v_caches[l]) for l in range(L)]
+    kn = [dev_u16_as_bf16(k_news[l]) for l in range(L)]
+    vn = [dev_u16_as_bf16(v_news[l]) for l in range(L)]
+    pl = to_dev(np.asarray(prefix_len, np.int32))
+    i32 = dict(dtype=torch.int32, device=DEV)
+    outs = dict(accept_len=torch.full((B,), -7, **i32), resampled=torch.full((B,), -7, **i32),
+                tokens=torch.full((B, k), -7, **i32), n_emitted=torch.full((B,), -7, **i32),
+                logp_d=torch.zeros((B, k), dtype=torch.float32, device=DEV),
+                logq_d=torch.zeros((B, k), dtype=torch.float32, device=DEV),
+                next_drafts=torch.full((B, k), -7, **i32),
+                next_preaccepted=torch.full((B,), 7, dtype=torch.uint8, device=DEV),
+                next_q_group=torch.full((B,), -7, **i32))
+    ws = workspace(abi.tidar_verify_commit_workspace_size(B, k, V))
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = outs
+    abi.tidar_verify_commit(p, q, dt, to_dev(inp["drafts"].astype(np.int32)),
+                            to_dev(inp["preaccepted"].astype(np.uint8)), to_dev(inp["u_acc"].astype(np.float32)),
+                            to_dev(inp["u_res"].astype(np.float32)), trust_ar, abi.pointer_array(kc, DEV),
+                            abi.pointer_array(vc, DEV), abi.pointer_array(kn, DEV), abi.pointer_array(vn, DEV), None, 0,
+                            0, L, B, Hkv, D, k, P_max, V, pl, g, to_dev(inp["u_draft"].astype(np.float32)),
+                            o["accept_len"], o["resampled"], o["tokens"], o["n_emitted"], o["logp_d"], o["logq_d"],
+                            o["next_drafts"], o["next_preaccepted"], o["next_q_group"], ws, ws.numel(), st)
+    torch.cuda.synchronize()
+
+    def back(ts):
+        return np.stack([t.view(torch.int16).cpu().numpy().view(np.uint16) for t in ts])
+
+    res = {n: t.cpu().numpy() for n, t in outs.items()}
+    res.update(k_caches=back(kc), v_caches=back(vc), prefix_len=pl.cpu().numpy(), status=int(st.item()))
+    if not want_status:
+        assert res["status"] == 0, f"device status {res['status']}"
+    return res
