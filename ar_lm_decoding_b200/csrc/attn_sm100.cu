@@ -29,7 +29,10 @@
 //               mask is evaluated from indices.
 //   warps 2-11  also load Q when its rows cannot come through TMA.
 // TMEM (512 columns): S buffers at [0, 128), [128, 256), [256, 384); O at
-// [384, 384+D).  P (bf16) overwrites the first 64 columns of its S buffer.
+// [384, 384+D).  P (bf16) overwrites columns [32, 96) of its S buffer: the P of
+// warpgroup w's keys lands in [32 + 32w, 64 + 32w), inside the columns that
+// warpgroup w itself read, so neither warpgroup can overwrite scores the other
+// has yet to load.
 // QK(j) reuses the buffer that PV(j-3) reads and is issued once PV(j-3) has
 // completed, so the softmax always has the next two tiles' S ready.
 // At the end each warpgroup reads its half of the columns of O and forms one
@@ -142,7 +145,10 @@ __device__ __forceinline__ void issue_qk(uint32_t d_s, uint64_t dq, uint64_t dk,
     }
 }
 
-// O(tmem) (+)= P(tmem) V: TN/16 MMAs over the keys.  P occupies the first TN/2 columns of S (two bf16 per
+// First TMEM column of P inside its S buffer (P of 128 keys: 64 columns, two bf16 per column).
+constexpr uint32_t kPCol = 32;
+
+// O(tmem) (+)= P(tmem) V: TN/16 MMAs over the keys.  P occupies TN/2 columns of S from kPCol (two bf16 per
 // column); V is MN-major, a 16-key step is 16 rows x 128 B (+128 in the descriptor's address field).
 template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t d_o, uint32_t a_p, uint64_t dv, uint32_t id, bool acc) {
@@ -529,7 +535,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                          tc::mbar_wait(p_full(sb), (i / 3) & 1, abort_flag, wl);
                     if (!ok) break;
                     tc::fence_after_sync();
-                    issue_pv<D>(tb + 384, tb + sb * 128, dv + vst * kStage, id_pv, i > 0);
+                    issue_pv<D>(tb + 384, tb + sb * 128 + kPCol, dv + vst * kStage, id_pv, i > 0);
                     tc::mma_commit(v_empty(vst));
                     tc::mma_commit(pv_done(i & 1));
                     if (i == n - 1) tc::mma_commit(o_final);
@@ -598,7 +604,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ghi = min(ghi, end);
             }
             float x[64];
-            const uint32_t pcol = s_col + w * 32;  // P of keys [64w, 64w+64) over S columns [32w, 32w+32)
+            // P of keys [64w, 64w+64) over S columns [32 + 32w, 64 + 32w): inside this warpgroup's own scores
+            const uint32_t pcol = s_col + kPCol + w * 32;
             const bool fresh = m_run == -INFINITY;  // no visible key so far: no max to reuse
             float hmx = -INFINITY, lt = 0.f;
             if (ok) {
