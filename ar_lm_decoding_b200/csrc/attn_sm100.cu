@@ -321,7 +321,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
     const int split = blockIdx.x, mt = blockIdx.y, bh = blockIdx.z;
-    const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+    const int kvh = bh % p.Hkv;
+    int b = bh / p.Hkv;  // (several sequences without splits: reassigned below, longest first)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long wl = p.wait_cycles;
     const int S = p.n_splits;  // cluster size; this CTA's rank is `split`
@@ -358,6 +359,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
     // every global read below (prefix lengths, Q, K/V) waits for the previous kernel
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
+    if (p.B > 1 && S == 1) {
+        // Several sequences and more row tiles than one wave holds: CTAs are dispatched in grid order, so the
+        // r-th group of KV heads takes the sequence with the r-th longest prefix (ties by index).  The first
+        // wave runs the longest, and the shortest fill the SMs that free up first.
+        int *seq_slot = reinterpret_cast<int *>(smem + L::MISC_OFF + 8);
+        const int rank_want = bh / p.Hkv;
+        for (int cand = tid; cand < p.B; cand += THREADS) {
+            const int pc = p.prefix_len[cand];
+            int rank = 0;
+            for (int o = 0; o < p.B; ++o) {
+                const int po = p.prefix_len[o];
+                rank += (po > pc) || (po == pc && o < cand);
+            }
+            if (rank == rank_want) *seq_slot = cand;
+        }
+        __syncthreads();
+        b = *seq_slot;
+    }
     if (tid == 0) {
         // Q does not depend on the prefix length: its copy starts at once
         if (q_tma) {  // rows (r, g) of the tile: box {64 d, G heads, 128/G rows}

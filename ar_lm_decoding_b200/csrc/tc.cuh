@@ -24,17 +24,17 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }
-// try_wait with a suspend-time hint: a waiting thread sleeps until the phase
-// completes (or ~1 ms passes) instead of spinning, so waiting warps leave
-// their scheduler's issue slots to the warps that compute.
+// try_wait without a suspend-time hint: the thread may wait in hardware for a
+// system-dependent time before the call returns false (measured: ~1 % faster
+// attention than a 1 ms hint, whose sleeping waiters wake later).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred P1;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
         "selp.b32 %0, 1, 0, P1;\n\t}\n"
         : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
 }
