@@ -50,9 +50,10 @@
 //
 // Before the previous kernel in the stream has finished (programmatic
 // dependent launch), a CTA sets up its barriers, tensor maps and TMEM; every
-// global read (prefix lengths, Q, K/V) waits for that kernel.  The first
-// tiles are then requested K, V, K, V, ... so the first PV's operand is not
-// queued behind every K stage.
+// global read (prefix lengths, Q, K/V) waits for that kernel.  Then only the
+// first QK's operands (Q and K of the first tile) are requested; the
+// producers stream V and the later tiles once that K has landed, so it is
+// not queued behind the start-up burst of every CTA (~20 MB at once).
 //
 // Every wait is bounded (p.wait_cycles).  On expiry the CTA raises
 // TIDAR_DEV_TIMEOUT in dev_status and every role stops; then the producers
@@ -454,14 +455,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     };
 
-    // ---- thread 0 starts the first copies at once ----
-    const int prologue = min(n, STAGES);
-    if (tid == 0) {
-        for (int i = 0; i < prologue; ++i) {
-            issue_tile(i, 0);
-            issue_tile(i, 1);
-        }
-    }
+    // ---- thread 0 starts the first K tile's copy at once; the producers stream the rest once it has landed ----
+    if (tid == 0 && n > 0) issue_tile(0, 0);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -491,8 +486,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             // ================= TMA producers: warp 0 streams K, warp 2 streams V =================
             const int is_v = warp == 2;
             if (lane == 0) {
-                int issued = prologue;
-                for (int i = prologue; i < n; ++i) {
+                // the first QK's operands (Q, K of tile 0) are served ahead of the rest of every CTA's burst
+                const int first = is_v ? 0 : min(n, 1);
+                int issued = first;
+                const bool k0_in = n == 0 || tc::mbar_wait(k_full(0), 0, abort_flag, wl);
+                for (int i = first; i < n && k0_in; ++i) {
                     const int u = i / STAGES;
                     if (!tc::mbar_wait(is_v ? v_empty(i % STAGES) : k_empty(i % STAGES), (u - 1) & 1, abort_flag, wl))
                         break;
