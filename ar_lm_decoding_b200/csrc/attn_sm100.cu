@@ -36,17 +36,19 @@
 // QK(j) reuses the buffer that PV(j-3) reads and is issued once PV(j-3) has
 // completed, so the softmax always has the next two tiles' S ready.
 // At the end each warpgroup reads its half of the columns of O and forms one
-// normalised partial row per query row, stored as fp16 with a per-half-row
-// fp32 scale (|error| <= 2^-12 of the row maximum) and its log2 LSE in fp32.
-// With one split that row is the output.  Otherwise the CTAs that split one
-// row tile's keys form a thread-block cluster: each CTA stages its records in
-// its own (idle) K/V ring, in the layout of the block every owner receives,
-// and sends each owner its block with one shared-to-shared bulk copy that
-// counts the bytes on the owner's receive barrier (armed at set-up); every
-// CTA merges its slice of rows over the S blocks (LSE weights, fixed order)
-// as soon as they have all landed, and writes the final bf16 output and LSE.
-// The cluster barrier has two phases: every CTA's ring is idle (waited for
-// before sending), and every CTA has received its blocks (before exit).
+// partial row per query row: the half row over its largest magnitude, stored
+// as fp16 (|error| <= 2^-12 of that magnitude), with an fp32 scale (that
+// magnitude over the row sum) and the row's log2 LSE in fp32.  With one split
+// the normalised row is the output.  Otherwise the CTAs that split one row
+// tile's keys form a thread-block cluster: each CTA stages its records in its
+// own (idle) K/V ring, in the layout of the block every owner receives, and
+// sends each owner its block with one shared-to-shared bulk copy that counts
+// the bytes on the owner's receive barrier (armed at set-up); every CTA merges
+// its slice of rows over the S blocks (LSE weights, fixed order) as soon as
+// they have all landed, and writes the final bf16 output and LSE.  One cluster
+// barrier (every CTA's ring is idle) comes before the copies; a CTA exits once
+// every other CTA has told it (a remote arrival on its "sent" barrier) that
+// all its blocks have landed, so no copy still reads its shared memory.
 //
 // Before the previous kernel in the stream has finished (programmatic
 // dependent launch), a CTA sets up its barriers, tensor maps and TMEM; every
@@ -105,8 +107,8 @@ struct Smem {
     static constexpr int STAGE_OFF = RECV_OFF + xchg_region_max(D);  // staged outgoing blocks (idem)
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
     // k_full, k_empty, v_full, v_empty, s_full[3], p_full[3], pv_done[2], o_final, q_full, fin_qk, fin_pv, stall,
-    // recv
-    static constexpr int NBARS = 4 * STAGES + 14;
+    // recv, sent
+    static constexpr int NBARS = 4 * STAGES + 15;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int XM_OFF = MISC_OFF + 16;  // row-max exchange between the warpgroups: [2][2][TM] bf16
     static constexpr int TOTAL = XM_OFF + 2 * 2 * TM * 2;
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t fin_pv = bar0 + 8u * (4 * STAGES + 11);  // the PV issuer's MMAs have all completed
     const uint32_t stall = bar0 + 8u * (4 * STAGES + 12);   // nothing arrives here (timeout test)
     const uint32_t recv = bar0 + 8u * (4 * STAGES + 13);    // every CTA's block of this CTA's rows has landed
+    const uint32_t sent = bar0 + 8u * (4 * STAGES + 14);    // every other CTA has received this CTA's block
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -347,6 +350,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::mbar_init(fin_pv, 1);
         tc::mbar_init(stall, 1);
         tc::mbar_init(recv, 1);
+        tc::mbar_init(sent, S > 1 ? S - 1 : 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
         // armed now with the bytes it is to receive (one block from every CTA of the cluster, itself included):
@@ -709,13 +713,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::fence_after_sync();
         // this CTA's ring is idle (every PV has read its V): first phase of the cluster barrier
         tc::cluster_arrive_relaxed();
-        // the row sum is split over the two halves
-        float *xl = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM] in the row-statistics area
-        xl[w * TM + row] = l_run;
-        asm volatile("bar.sync 1, 256;\n" ::: "memory");
-        const float ltot = l_run + xl[(1 - w) * TM + row];
-        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-        const float lse2 = ltot > 0.f ? m_run + __log2f(ltot) : -INFINITY;  // log2 of this CTA's row sum
+        // this half row of O (its copy from TMEM overlaps the row-sum exchange below)
         uint32_t va[H / 32][32];
 #pragma unroll
         for (int c = 0; c < H / 32; ++c) {
@@ -723,14 +721,22 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int j = 0; j < 32; ++j) va[c][j] = 0u;
             if (fin) tc::tmem_ld32(o_col + c * 32, va[c]);
         }
+        // the row sum is split over the two halves
+        float *xl = reinterpret_cast<float *>(smem + L::KV_OFF);  // [2][TM] in the row-statistics area
+        xl[w * TM + row] = l_run;
+        asm volatile("bar.sync 1, 256;\n" ::: "memory");
+        const float ltot = l_run + xl[(1 - w) * TM + row];
+        const float inv = ltot > 0.f ? __fdividef(1.f, ltot) : 0.f;
+        const float lse2 = ltot > 0.f ? m_run + __log2f(ltot) : -INFINITY;  // log2 of this CTA's row sum
         tc::tmem_wait_ld();
-        float hv[H];
-#pragma unroll
-        for (int c = 0; c < H / 32; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) hv[c * 32 + j] = fin ? __uint_as_float(va[c][j]) * inv : 0.f;
+        tc::fence_before_sync();  // (TMEM is freed after a later barrier)
         if (S == 1) {  // the CTA saw every key of its rows: the normalised half row is the output
             if (m_row < p.M) {
+                float hv[H];
+#pragma unroll
+                for (int c = 0; c < H / 32; ++c)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) hv[c * 32 + j] = __uint_as_float(va[c][j]) * inv;
                 const size_t orow = (size_t)(b * p.R + r) * p.Hq + kvh * p.G + (m_row - r * p.G);
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + w * H);
 #pragma unroll
@@ -741,23 +747,27 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             tc::cluster_wait();  // (first phase)
         } else {
-            // this row's record, staged in this CTA's (idle) ring in the layout of the block its owner receives
+            // this row's record, staged in this CTA's (idle) ring in the layout of the block its owner receives:
+            // the unnormalised half row over its largest magnitude (so in [-1, 1]), and that magnitude / the row sum
             float am[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-            for (int j = 0; j < H; ++j) am[j & 3] = fmaxf(am[j & 3], fabsf(hv[j]));
+            for (int j = 0; j < H; ++j) am[j & 3] = fmaxf(am[j & 3], fabsf(__uint_as_float(va[j >> 5][j & 31])));
             const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
-            const float scale = amax > 0.f ? amax : 1.f;  // stored values are hv / scale, in [-1, 1]
-            const float rs = 1.f / scale;
+            const float rs = amax > 0.f ? __fdividef(1.f, amax) : 0.f;
+            const float scale = amax * inv;  // the stored value times this is the normalised one
             const int per = xchg_per(S), pv = per | 1;
             const int VB = xchg_vals_bytes(S, D), BB = xchg_block_bytes(S, D);
             const int owner = row / per, rl = row - owner * per;
             uint8_t *stage = smem + L::STAGE_OFF;  // [owner][vals | hdr]
             uint4 *vals = reinterpret_cast<uint4 *>(stage + owner * BB);
 #pragma unroll
-            for (int j = 0; j < H / 8; ++j)
-                vals[(w * (H / 8) + j) * pv + rl] =
-                    make_uint4(pack_half2(hv[8 * j] * rs, hv[8 * j + 1] * rs), pack_half2(hv[8 * j + 2] * rs, hv[8 * j + 3] * rs),
-                               pack_half2(hv[8 * j + 4] * rs, hv[8 * j + 5] * rs), pack_half2(hv[8 * j + 6] * rs, hv[8 * j + 7] * rs));
+            for (int j = 0; j < H / 8; ++j) {
+                float o8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o8[e] = __uint_as_float(va[(8 * j + e) >> 5][(8 * j + e) & 31]) * rs;
+                vals[(w * (H / 8) + j) * pv + rl] = make_uint4(pack_half2(o8[0], o8[1]), pack_half2(o8[2], o8[3]),
+                                                               pack_half2(o8[4], o8[5]), pack_half2(o8[6], o8[7]));
+            }
             float *hdr = reinterpret_cast<float *>(stage + owner * BB + VB) + rl * 4;
             hdr[1 + w] = scale;
             if (w == 0) hdr[0] = lse2;
@@ -777,6 +787,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool got = tc::mbar_wait_drain(recv, 0, kDrainCycles);
         if (!got && tid == 0) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
         if (__syncthreads_and(got)) {
+            // every other CTA's copy into this CTA has completed, so its source block has been read: each source
+            // hears of it at once (lane o of warp 0 tells CTA o; it may exit once all its blocks are in)
+            if (warp == 0 && lane < S && lane != split) tc::mbar_arrive_remote(tc::cluster_map(sent, lane));
             const uint8_t *rv = smem + L::RECV_OFF;
             float *wts = reinterpret_cast<float *>(smem + L::KV_OFF);  // row-statistics area, free by now
             switch (S) {
@@ -790,10 +803,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     }
-    // second phase of the cluster barrier: every CTA has received all its blocks, so no copy is in flight into
-    // or out of any CTA of the cluster when it exits
-    tc::cluster_arrive_relaxed();
-    tc::cluster_wait();
+    if (S > 1) {
+        // no copy may still read this CTA's shared memory when it exits: wait until every block it sent has landed
+        if (tid == 0 && !tc::mbar_wait_drain(sent, 0, kDrainCycles)) atomicOr(p.dev_status, TIDAR_DEV_TIMEOUT);
+    } else {
+        // (a cluster of one: every thread is past its TMEM reads before the allocation is freed)
+        tc::cluster_arrive_relaxed();
+        tc::cluster_wait();
+    }
     if (warp == 1) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tbase, 512);

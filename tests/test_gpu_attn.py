@@ -112,6 +112,40 @@ def test_running_max_growth_rescales(B, Hq, Hkv, P):
     _check_full(cfg, inp=inp)
 
 
+def _plant_deep_first_tiles(cfg, inp, depth_nat=100.0):
+    """For every KV head and every even 128-key tile t of the cache (with a tile after it), pull all keys of
+    tile t, and the keys in columns 64..127 of tile t+1, away from one query row of that head's group, so that
+    the row scores about -depth_nat natural-log units there.  A CTA that meets tile t first sets that row's
+    running max ~depth_nat / ln 2 log2-units below the scores of tile t+1's first half: exponentials against
+    the stale max overflow there (in one column half only) before the row's max is renewed."""
+    q = synth.bf16_bits_to_f32(inp["q"]).astype(np.float64)
+    kc = synth.bf16_bits_to_f32(inp["k_cache"]).astype(np.float64)
+    G = cfg.Hq // cfg.Hkv
+    scale = 1.0 / np.sqrt(cfg.D)
+    for b in range(cfg.B):
+        P = int(inp["prefix_len"][b])
+        nt = (P + 127) // 128
+        for h in range(cfg.Hkv):
+            for t in range(0, nt - 1, 2):
+                r, g = t % cfg.R, h * G + (t // 2) % G
+                qv = q[b, r, g]
+                alpha = depth_nat / (scale * float(qv @ qv))
+                for n in list(range(t * 128, t * 128 + 128)) + list(range(t * 128 + 192, t * 128 + 256)):
+                    if n < P:
+                        kc[b, h, n] = kc[b, h, n] - alpha * qv
+    out = dict(inp)
+    out["k_cache"] = synth.f32_to_bf16_bits(kc.astype(np.float32))
+    return out
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,P", [(1, 8, 2, 2000), (2, 4, 1, 1200)])
+def test_running_max_jump_beyond_float_range(B, Hq, Hkv, P):
+    # a row's max jumps by ~144 log2-units from one tile to the next (2^144 overflows fp32 and bf16)
+    cfg = TINY.with_(B=B, Hq=Hq, Hkv=Hkv, D=128, k=3, P=P)
+    inp = _plant_deep_first_tiles(cfg, synth.make_attn_inputs(cfg, seed=11))
+    _check_full(cfg, inp=inp)
+
+
 def test_group_rows_ignore_later_drafts_bitwise():
     cfg = TINY.with_(k=4, P=190, Hq=4, Hkv=2)
     k = cfg.k
