@@ -35,6 +35,8 @@
 // has yet to load.
 // QK(j) reuses the buffer that PV(j-3) reads and is issued once PV(j-3) has
 // completed, so the softmax always has the next two tiles' S ready.
+// The S CTAs of a row tile take its key tiles round robin (split s: tiles s,
+// s + S, ...), so that a split's first tile does not depend on the prefix.
 // At the end each warpgroup reads its half of the columns of O and forms one
 // partial row per query row: the half row over its largest magnitude, stored
 // as fp16 (|error| <= 2^-12 of that magnitude), with an fp32 scale (that
@@ -53,9 +55,11 @@
 // Before the previous kernel in the stream has finished (programmatic
 // dependent launch), a CTA sets up its barriers, tensor maps and TMEM; every
 // global read (prefix lengths, Q, K/V) waits for that kernel.  Then only the
-// first QK's operands (Q and K of the first tile) are requested; the
-// producers stream V and the later tiles once that K has landed, so it is
-// not queued behind the start-up burst of every CTA (~20 MB at once).
+// first QK's operands (Q and K of the first tile) are requested -- with a
+// contiguous cache both at once, before the prefix length is known (the K
+// copy is dropped if the prefix ends before that tile); the producers stream
+// V and the later tiles once that K has landed, so it is not queued behind
+// the start-up burst of every CTA (~20 MB at once).
 //
 // Every wait is bounded (p.wait_cycles).  On expiry the CTA raises
 // TIDAR_DEV_TIMEOUT in dev_status and every role stops; then the producers
@@ -107,8 +111,8 @@ struct Smem {
     static constexpr int STAGE_OFF = RECV_OFF + xchg_region_max(D);  // staged outgoing blocks (idem)
     static constexpr int BAR_OFF = KV_OFF + STAGES * STAGE;
     // k_full, k_empty, v_full, v_empty, s_full[3], p_full[3], pv_done[2], o_final, q_full, fin_qk, fin_pv, stall,
-    // recv, sent
-    static constexpr int NBARS = 4 * STAGES + 15;
+    // recv, sent, k_spec
+    static constexpr int NBARS = 4 * STAGES + 16;
     static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
     static constexpr int XM_OFF = MISC_OFF + 16;  // row-max exchange between the warpgroups: [2][2][TM] bf16
     static constexpr int TOTAL = XM_OFF + 2 * 2 * TM * 2;
@@ -285,12 +289,13 @@ __device__ __forceinline__ int tile_valid(int t, int TP, int P, int R) {
     return t < TP ? min(TN, P - t * TN) : min(TN, R - (t - TP) * TN);
 }
 
-// Key tiles [t0, t1) of split `split` out of n_splits for a sequence with prefix length P.
-__device__ __forceinline__ void split_range(int P, int R, int split, int n_splits, int &TP, int &t0, int &t1) {
+// Key tiles of split `split` out of n_splits for a sequence with prefix length P (TP prefix tiles, then the
+// new-key tiles): tiles split, split + n_splits, split + 2 n_splits, ... -- n of them.  Round robin, so that a
+// split's first tile does not depend on P.
+__device__ __forceinline__ void split_tiles(int P, int R, int split, int n_splits, int &TP, int &n) {
     TP = ceil_div(P, TN);
     const int T = TP + ceil_div(R, TN);
-    t0 = (int)((long)split * T / n_splits);
-    t1 = (int)((long)(split + 1) * T / n_splits);
+    n = split < T ? (T - split + n_splits - 1) / n_splits : 0;
 }
 
 template <int D>
@@ -321,6 +326,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t stall = bar0 + 8u * (4 * STAGES + 12);   // nothing arrives here (timeout test)
     const uint32_t recv = bar0 + 8u * (4 * STAGES + 13);    // every CTA's block of this CTA's rows has landed
     const uint32_t sent = bar0 + 8u * (4 * STAGES + 14);    // every other CTA has received this CTA's block
+    const uint32_t k_spec = bar0 + 8u * (4 * STAGES + 15);  // the early copy of cache tile `split` (below)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF + 4);
 
@@ -351,6 +357,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::mbar_init(stall, 1);
         tc::mbar_init(recv, 1);
         tc::mbar_init(sent, S > 1 ? S - 1 : 1);
+        tc::mbar_init(k_spec, 1);
         *abort_flag = 0;
         tc::mbar_fence_init();
         // armed now with the bytes it is to receive (one block from every CTA of the cluster, itself included):
@@ -391,10 +398,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc::tma_load_3d(sQ + h * TM * 128, &tm_q, h * 64, kvh * p.G, b * p.R + mt * (TM / p.G), q_full);
         }
     }
+    // With a contiguous cache the first tile of this split, cache tile `split`, does not depend on the prefix
+    // length either: its copy starts now too, into the K slot of the ring's last stage, counted on k_spec.  If the
+    // prefix reaches that tile it is kept, and tile i of the split goes to stage (i + STAGES - 1) % STAGES;
+    // otherwise tile i goes to stage i % STAGES, and the last stage is reused only once the copy has landed.
+    // (Rows past the cache read as zeros.)
+    const bool spec = !p.block_table;
+    if (tid == 0 && spec) {
+        tc::mbar_arrive_expect_tx(k_spec, L::KV_TILE);
+        const int y = (b * p.Hkv + kvh) * p.P_max + split * TN;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+            tc::tma_load_2d(sKV + (STAGES - 1) * L::STAGE + h * TN * 128, &tm_kc, h * 64, y, k_spec);
+    }
     const int P = p.prefix_len[b];
-    int TP = 0, t0 = 0, t1 = 0;
+    int TP = 0, n = 0;
     const bool bad_prefix = P < 0 || P > p.P_max;
-    if (!bad_prefix) split_range(P, p.R, split, S, TP, t0, t1);
+    if (!bad_prefix) split_tiles(P, p.R, split, S, TP, n);
+    const bool spec_ok = spec && n > 0 && split < TP;  // the early copy is this split's first tile
+    const int so = spec_ok ? STAGES - 1 : 0;             // tile i of the split uses ring stage (i + so) % STAGES
     bool bad_page = false;
     if (p.block_table && !bad_prefix) {  // (uniform over the CTA: one sequence)
         // every CTA of the cluster checks every page of the sequence, so that they all take the same exit (the
@@ -412,6 +434,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (tid == 0 && split == 0 && mt == 0)
             atomicOr(p.dev_status, bad_prefix ? TIDAR_DEV_BAD_PREFIX : TIDAR_DEV_BAD_PAGE);
         if (tid == 0 && q_tma) tc::mbar_wait_drain(q_full, 0, kDrainCycles);  // no copy may land after exit
+        if (tid == 0 && spec) tc::mbar_wait_drain(k_spec, 0, kDrainCycles);
         tc::fence_before_sync();
         __syncthreads();
         if (warp == 1) {
@@ -420,7 +443,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         return;
     }
-    const int n = t1 - t0;
     // cache row of box h2 (0, 1: the two 64-row halves) of cache tile t: contiguous, or through the block table
     // (read as the copy is issued; the table is not written during the launch).  The second box of a last tile
     // that ends within its first page has no page of its own: it re-reads the first page (rows past P are
@@ -432,12 +454,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         return (pg * p.Hkv + kvh) * BOXR;
     };
 
-    // K (is_v = 0) or V (is_v = 1) of tile i into stage i % STAGES of its ring: two 64-row boxes per column block
+    // K (is_v = 0) or V (is_v = 1) of tile i into stage (i + so) % STAGES of its ring
     auto issue_tile = [&](int i, int is_v) {
-        const int st = i % STAGES;
+        const int st = (i + so) % STAGES;
         const uint32_t bar = is_v ? v_full(st) : k_full(st);
         tc::mbar_arrive_expect_tx(bar, L::KV_TILE);
-        const int t = t0 + i;
+        const int t = split + i * S;
         const uint32_t dst = sKV + st * L::STAGE + is_v * L::KV_TILE;
         if (t < TP && p.block_table) {  // two 64-row boxes, one per page
 #pragma unroll
@@ -459,8 +481,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     };
 
-    // ---- thread 0 starts the first K tile's copy at once; the producers stream the rest once it has landed ----
-    if (tid == 0 && n > 0) issue_tile(0, 0);
+    // ---- the first K tile's copy (paged cache: starts now); the producers stream the rest once it has landed ----
+    if (tid == 0 && n > 0 && !spec_ok) issue_tile(0, 0);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -493,20 +515,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // the first QK's operands (Q, K of tile 0) are served ahead of the rest of every CTA's burst
                 const int first = is_v ? 0 : min(n, 1);
                 int issued = first;
-                const bool k0_in = n == 0 || tc::mbar_wait(k_full(0), 0, abort_flag, wl);
+                // (kept early copy: it completes the last stage's first K phase; the QK of tile 0 waits on k_spec)
+                if (!is_v && spec_ok) tc::mbar_arrive(k_full(so));
+                const bool k0_in = n == 0 || tc::mbar_wait(spec_ok ? k_spec : k_full(0), 0, abort_flag, wl);
                 for (int i = first; i < n && k0_in; ++i) {
                     const int u = i / STAGES;
-                    if (!tc::mbar_wait(is_v ? v_empty(i % STAGES) : k_empty(i % STAGES), (u - 1) & 1, abort_flag, wl))
-                        break;
+                    const int st = (i + so) % STAGES;
+                    if (!tc::mbar_wait(is_v ? v_empty(st) : k_empty(st), (u - 1) & 1, abort_flag, wl)) break;
+                    // (a dropped early copy: the last stage's K slot is rewritten once it has landed)
+                    if (!is_v && spec && !spec_ok && st == STAGES - 1 && u == 0)
+                        tc::mbar_wait_drain(k_spec, 0, kDrainCycles);
                     issue_tile(i, is_v);
                     issued = i + 1;
                 }
                 // drain, whatever happened: only the last copy of each stage can still be in flight (an earlier
                 // one completed before its stage was re-armed), and none may land after the CTA exits
                 for (int i = max(0, issued - STAGES); i < issued; ++i)
-                    tc::mbar_wait_drain(is_v ? v_full(i % STAGES) : k_full(i % STAGES), (i / STAGES) & 1,
+                    tc::mbar_wait_drain(is_v ? v_full((i + so) % STAGES) : k_full((i + so) % STAGES), (i / STAGES) & 1,
                                         kDrainCycles);
                 if (!is_v && q_tma) tc::mbar_wait_drain(q_full, 0, kDrainCycles);
+                if (!is_v && spec) tc::mbar_wait_drain(k_spec, 0, kDrainCycles);
             }
             __syncwarp();
         } else {
@@ -523,24 +551,19 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint64_t dk = tc::smem_desc_sw128(sKV, 16, 1024);
                 bool ok = !p.stall_test || tc::mbar_wait(stall, 0, abort_flag, wl);
                 ok = ok && tc::mbar_wait(q_full, 0, abort_flag, wl);
-                int kst = 0;
-                uint32_t kph = 0;
                 for (int j = 0; j < n && ok; ++j) {
-                    const int sb = j % 3;
+                    const int sb = j % 3, kst = (j + so) % STAGES;
+                    const uint32_t kph = (j / STAGES) & 1;
                     if (j >= 3) {  // PV(j-3) done reading P from buffer sb (PV(j-5) was waited for before)
                         ok = tc::mbar_wait(pv_done((j - 3) & 1), ((j - 3) >> 1) & 1, abort_flag, wl);
                         if (!ok) break;
                     }
-                    ok = tc::mbar_wait(k_full(kst), kph, abort_flag, wl);
+                    ok = tc::mbar_wait(j == 0 && spec_ok ? k_spec : k_full(kst), kph, abort_flag, wl);
                     if (!ok) break;
                     tc::fence_after_sync();
                     issue_qk<D>(tb + sb * 128, dq, dk + kst * kStage, id_qk);
                     tc::mma_commit(s_full(sb));
                     tc::mma_commit(k_empty(kst));
-                    if (++kst == STAGES) {
-                        kst = 0;
-                        kph ^= 1u;
-                    }
                 }
                 tc::mma_commit(fin_qk);  // every MMA of this thread completes before TMEM is freed
                 tc::mbar_wait_drain(fin_qk, 0, kDrainCycles);
@@ -548,10 +571,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 constexpr uint32_t id_pv = tc::idesc_bf16_f32(TM, D, 0, 1);
                 const uint64_t dv = tc::smem_desc_sw128(sKV + L::KV_TILE, TN * 128, 1024);
                 bool ok = true;
-                int vst = 0;
-                uint32_t vph = 0;
                 for (int i = 0; i < n && ok; ++i) {
-                    const int sb = i % 3;
+                    const int sb = i % 3, vst = (i + so) % STAGES;
+                    const uint32_t vph = (i / STAGES) & 1;
                     ok = tc::mbar_wait(v_full(vst), vph, abort_flag, wl) &&
                          tc::mbar_wait(p_full(sb), (i / 3) & 1, abort_flag, wl);
                     if (!ok) break;
@@ -560,10 +582,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc::mma_commit(v_empty(vst));
                     tc::mma_commit(pv_done(i & 1));
                     if (i == n - 1) tc::mma_commit(o_final);
-                    if (++vst == STAGES) {
-                        vst = 0;
-                        vph ^= 1u;
-                    }
                 }
                 tc::mma_commit(fin_pv);
                 tc::mbar_wait_drain(fin_pv, 0, kDrainCycles);
@@ -605,7 +623,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             bool have = ok && tc::mbar_wait(s_full(sb), (i / 3) & 1, abort_flag, wl);
             ok = __all_sync(0xffffffffu, have);  // TMEM accesses are warp-collective: decide per warp
             const uint32_t s_col = tbase + lane_off + sb * 128;
-            const int t = t0 + i;
+            const int t = split + i * S;
             // a partial prefix tile (keys beyond P) or a new-key tile (the TiDAR mask): the visible keys of
             // this row are [0, lo) and [glo, ghi); everything else, garbage included, is excluded by select
             const bool masked = t >= TP - 1 && !(t == TP - 1 && P % TN == 0);
@@ -687,7 +705,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int valid = tile_valid(t, TP, P, p.R);
             if (ok && valid < TN) {
                 // keys past the sequence: zero their V rows (0 * garbage could be NaN) before PV reads them
-                const int st = i % STAGES;
+                const int st = (i + so) % STAGES;
                 const bool got = tc::mbar_wait(v_full(st), (i / STAGES) & 1, abort_flag, wl);
                 ok = __all_sync(0xffffffffu, got);
                 if (ok) {
