@@ -85,10 +85,11 @@ static_assert(BOXR == kPageRows, "a TMA box of the cache is one page");
 
 // Split-KV exchange of an S-CTA cluster.  CTA s merges rows [s*per, (s+1)*per) of the row tile, per =
 // ceil(128 / S).  Every CTA sends each owner one block with its partial records of the owner's rows:
-//   vals [D/8][pv]  16-byte chunks (8 fp16 of one row, divided by the half-row scale), pv = per rounded up to an
-//                   odd number, so that reading one chunk of consecutive rows and reading the consecutive chunks
-//                   of one row both spread over all shared-memory banks
-//   hdr  [per]      float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused)
+//   vals [D/8][pv]  16-byte chunks (8 fp16 of one row, over its half row's largest magnitude), pv = per rounded
+//                   up to an odd number, so that reading one chunk of consecutive rows and reading the consecutive
+//                   chunks of one row both spread over all shared-memory banks
+//   hdr  [per]      float4 (log2 LSE, scale of columns [0, D/2), scale of [D/2, D), unused); a half's scale is
+//                   its largest magnitude over the row sum, so value x scale is the normalised partial output
 // The owner receives the S blocks in source order.  Both the received blocks and the staged outgoing ones live
 // in the CTA's K/V ring, which is idle by then: [row statistics | received | staged].
 __host__ __device__ constexpr int xchg_per(int S) { return (TM + S - 1) / S; }

@@ -611,13 +611,18 @@ def load_traffic(cfg):
 
 
 def kernel_source_hash():
+    """Hash of the attention kernel's code (its sources with comments and layout removed), so that the DRAM
+    traffic recorded for it is dropped when the code changes but kept across comment edits."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ar_lm_decoding_b200", "csrc")
     for n in sorted(os.listdir(csrc)):
         if n.startswith("attn") or n in ("common.cuh", "tc.cuh"):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(n.encode() + f.read())
+            with open(os.path.join(csrc, n)) as f:
+                code = re.sub(r"/\*.*?\*/", " ", f.read(), flags=re.S)
+            code = " ".join(re.sub(r"//[^\n]*", " ", code).split())
+            h.update(n.encode() + code.encode())
     return h.hexdigest()
 
 

@@ -94,8 +94,11 @@ size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max
  * q          bf16 [B, R, Hq, D]   post-RoPE queries
  * k_new      bf16 [B, R, Hkv, D]  post-RoPE keys of this step's R tokens
  * v_new      bf16 [B, R, Hkv, D]
- * k_cache    bf16 [B, Hkv, P_max, D]  rows 0..P_b-1 are read, nothing else
- * v_cache    bf16 [B, Hkv, P_max, D]
+ * k_cache    bf16 [B, Hkv, P_max, D]  rows 0..P_b-1 are used; whole 128-row tiles
+ *            are read (with a contiguous cache also up to 8 tiles from row 0
+ *            whatever P_b is), always inside the buffer, and rows past P_b are
+ *            ignored, whatever they hold (NaN included)
+ * v_cache    bf16 [B, Hkv, P_max, D]  (likewise)
  * prefix_len int32 [B]  P_b, 0 <= P_b <= P_max
  * Hq % Hkv == 0; query head h reads KV head h / (Hq/Hkv).  D in {64, 128}.
  * softmax_scale  score multiplier, > 0 (1/sqrt(D) for the standard scale).

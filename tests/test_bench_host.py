@@ -52,7 +52,7 @@ def test_traffic_figure_only_for_matching_sources(tmp_path, monkeypatch):
     csrc = tmp_path / "ar_lm_decoding_b200" / "csrc"
     csrc.mkdir(parents=True)
     for n in ("attn_sm100.cu", "attn.cuh", "common.cuh", "tc.cuh", "verify.cu"):
-        (csrc / n).write_text(f"// {n}\n")
+        (csrc / n).write_text(f"// {n}\nint x_{n.replace('.', '_')} = 1;\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     cfg = synth.CONFIGS["qwen3-8b_k8"]
@@ -61,9 +61,11 @@ def test_traffic_figure_only_for_matching_sources(tmp_path, monkeypatch):
     path.write_text(json.dumps(rec))
     assert bench.load_traffic(cfg) == 123
     assert bench.load_traffic(synth.CONFIGS["qwen2.5-1.5b_k4"]) is None  # another workload
-    (csrc / "verify.cu").write_text("// changed\n")  # not an attention source: the figure stands
+    (csrc / "verify.cu").write_text("int changed = 2;\n")  # not an attention source: the figure stands
     assert bench.load_traffic(cfg) == 123
-    (csrc / "tc.cuh").write_text("// changed\n")  # the attention kernel changed: no figure
+    (csrc / "tc.cuh").write_text("/* a new comment */ // and another\nint   x_tc_cuh =\n 1;\n")  # comments, layout
+    assert bench.load_traffic(cfg) == 123
+    (csrc / "tc.cuh").write_text("int x_tc_cuh = 2;\n")  # the attention kernel's code changed: no figure
     assert bench.load_traffic(cfg) is None
     path.write_text("{not json")
     assert bench.load_traffic(cfg) is None
