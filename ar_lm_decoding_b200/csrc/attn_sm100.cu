@@ -224,8 +224,8 @@ __device__ __forceinline__ float half_exp(uint32_t pcol, const float (&x)[64], f
 
 // Merge of this CTA's rows over the S blocks received (all THREADS threads).  First the weights of every row:
 // w_s = exp2(lse_s - max) / sum * scale_s per column half (in the row-statistics area, free by then); then items
-// (row, 16-byte column chunk), consecutive threads on consecutive chunks of one row, so that every warp writes
-// whole output rows.  Sources are summed in a fixed order.
+// (row, one 16-byte column chunk of each half), consecutive threads on consecutive chunks of one row, so that
+// every warp writes whole output rows in one round.  Sources are summed in a fixed order.
 template <int D, int S>
 __device__ __forceinline__ void merge_rows(const AttnParams &p, const uint8_t *recv, float *wts, int split, int mt,
                                            int b, int kvh, int tid) {
@@ -245,7 +245,7 @@ __device__ __forceinline__ void merge_rows(const AttnParams &p, const uint8_t *r
             wq[sp] = hd[sp].x == -INFINITY ? 0.f : fast_exp2(hd[sp].x - mx);
             wsum += wq[sp];
         }
-        const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+        const float winv = wsum > 0.f ? __fdividef(1.f, wsum) : 0.f;
         float *w = wts + rl * (2 * S + 2);
 #pragma unroll
         for (int sp = 0; sp < S; ++sp) {
@@ -255,31 +255,40 @@ __device__ __forceinline__ void merge_rows(const AttnParams &p, const uint8_t *r
         w[2 * S] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;  // natural-log LSE
     }
     __syncthreads();
-    for (int it = tid; it < nrows * CH; it += THREADS) {
-        const int rl = it / CH, c = it - rl * CH;
+    // items (row, chunk c of the first column half and chunk c + CH/2 of the second): one round for every row
+    constexpr int HC = CH / 2;
+    for (int it = tid; it < nrows * HC; it += THREADS) {
+        const int rl = it / HC, c = it - rl * HC;
         const float *w = wts + rl * (2 * S + 2);
-        float acc[8];
+        float acc[2][8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
 #pragma unroll
         for (int sp = 0; sp < S; ++sp) {
-            const uint4 raw = reinterpret_cast<const uint4 *>(recv + sp * BB)[c * pv + rl];
-            const float f = w[2 * sp + (c < CH / 2 ? 0 : 1)];
-            const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 v = unpack_half2(u[e]);
-                acc[2 * e] = fmaf(f, v.x, acc[2 * e]);
-                acc[2 * e + 1] = fmaf(f, v.y, acc[2 * e + 1]);
+            for (int h = 0; h < 2; ++h) {
+                const uint4 raw = reinterpret_cast<const uint4 *>(recv + sp * BB)[(c + h * HC) * pv + rl];
+                const float f = w[2 * sp + h];
+                const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 v = unpack_half2(u[e]);
+                    acc[h][2 * e] = fmaf(f, v.x, acc[h][2 * e]);
+                    acc[h][2 * e + 1] = fmaf(f, v.y, acc[h][2 * e + 1]);
+                }
             }
         }
         const int m = mt * TM + row0 + rl;
         if (m < p.M) {
             const int rq = m / p.G;
             const size_t orow = (size_t)(b * p.R + rq) * p.Hq + kvh * p.G + (m - rq * p.G);
-            *reinterpret_cast<uint4 *>(p.out + orow * D + c * 8) =
-                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                           pack_bf16x2(acc[6], acc[7]));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                *reinterpret_cast<uint4 *>(p.out + orow * D + (c + h * HC) * 8) =
+                    make_uint4(pack_bf16x2(acc[h][0], acc[h][1]), pack_bf16x2(acc[h][2], acc[h][3]),
+                               pack_bf16x2(acc[h][4], acc[h][5]), pack_bf16x2(acc[h][6], acc[h][7]));
             if (c == 0 && p.lse) p.lse[orow] = w[2 * S];
         }
     }
