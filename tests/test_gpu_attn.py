@@ -146,6 +146,21 @@ def test_running_max_jump_beyond_float_range(B, Hq, Hkv, P):
     _check_full(cfg, inp=inp)
 
 
+@pytest.mark.parametrize("seed", range(16))
+def test_random_shapes(seed):
+    """Seeded random shapes, every row against the oracle: batch 1..4 with ragged prefix lengths (short sequences
+    beside long ones in one launch, so splits whose first key tile lies past a short prefix sit next to splits
+    that keep it), 1..4 KV heads, group sizes 1..8, D 64 or 128, draft length 1..10, both mask modes."""
+    rng = np.random.default_rng(1000 + seed)
+    Hkv = int(rng.choice([1, 2, 4]))
+    G = int(rng.choice([1, 2, 3, 4, 8]))
+    hi = int(rng.integers(1, 2500))
+    cfg = TINY.with_(B=int(rng.integers(1, 5)), Hq=Hkv * G, Hkv=Hkv, D=int(rng.choice([64, 128])),
+                     k=int(rng.integers(1, 11)), P=hi, ragged=(0, hi))
+    mode = oracle.MASK_HYBRID if seed % 3 else oracle.MASK_CAUSAL
+    _check_full(cfg, seed=seed, mode=mode)
+
+
 def test_group_rows_ignore_later_drafts_bitwise():
     cfg = TINY.with_(k=4, P=190, Hq=4, Hkv=2)
     k = cfg.k
