@@ -536,14 +536,15 @@ def graph_us(stream, reps, fn):
     return e0.elapsed_time(e1) * 1e3 / reps
 
 
-def copy_groups(L):
-    """Layers per host-to-device copy in the end-to-end step: 1, 2, 4, ... (the last group takes the rest), so
-    that the first layer starts after one layer's inputs while the copies stay few (each copy costs a fixed
-    overhead: one per layer ran the Qwen3-8B inputs at 45 GB/s, groups of 12-18 layers at 51, of a 55 GB/s link)."""
+def copy_groups(L, cap=8):
+    """Layers per host-to-device copy in the end-to-end step: 1, 2, 4, 8, 8, ... (the last group takes the rest),
+    so that the first layer starts after one layer's inputs while the copies stay few (each copy costs a fixed
+    overhead: one per layer ran the Qwen3-8B inputs at 45 GB/s, groups of 6-18 layers at 50.6-51.4, of a 55 GB/s
+    link); the cap keeps a compute-bound step from waiting on one very large late copy."""
     groups, l0, n = [], 0, 1
     while l0 < L:
         groups.append((l0, min(L, l0 + n)))
-        l0, n = l0 + n, 2 * n
+        l0, n = l0 + n, min(cap, 2 * n)
     return groups
 
 
