@@ -673,7 +673,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             // is within 2^8 of the true maximum serves); every warp passes this barrier on every tile
             const __nv_bfloat16 hb = __float2bfloat16_rn(hmx);
             xm[((i & 1) * 2 + w) * TM + row] = hb;
-            asm volatile("bar.sync 1, 256;\n" ::: "memory");
+            // only the two warps that hold the two halves of these 32 rows (warps 4 + q4 and 8 + q4) meet here
+            asm volatile("bar.sync %0, 64;\n" ::"r"(2 + q4) : "memory");
             const __nv_bfloat16 ob = xm[((i & 1) * 2 + (1 - w)) * TM + row];
             if (ok) {
                 const float mx = fmaxf(__bfloat162float(hb), __bfloat162float(ob)) * sl2;
