@@ -482,7 +482,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else if (t < TP) {  // one 128-row box per column block
             const int y = (b * p.Hkv + kvh) * p.P_max + t * TN;
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) tc::tma_load_2d(dst + h * TN * 128, is_v ? &tm_vc : &tm_kc, h * 64, y, bar);
+            for (int h = 0; h < D / 64; ++h)
+                tc::tma_load_2d(dst + h * TN * 128, is_v ? &tm_vc : &tm_kc, h * 64, y, bar);
         } else {
             const int z = b * p.R + (t - TP) * TN;
 #pragma unroll
@@ -770,8 +771,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * D + w * H);
 #pragma unroll
                 for (int j = 0; j < H / 8; ++j)
-                    dst[j] = make_uint4(pack_bf16x2(hv[8 * j], hv[8 * j + 1]), pack_bf16x2(hv[8 * j + 2], hv[8 * j + 3]),
-                                        pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]), pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
+                    dst[j] = make_uint4(pack_bf16x2(hv[8 * j], hv[8 * j + 1]),
+                                        pack_bf16x2(hv[8 * j + 2], hv[8 * j + 3]),
+                                        pack_bf16x2(hv[8 * j + 4], hv[8 * j + 5]),
+                                        pack_bf16x2(hv[8 * j + 6], hv[8 * j + 7]));
                 if (w == 0 && p.lse) p.lse[orow] = lse2 * kLn2;
             }
             tc::cluster_wait();  // (first phase)
