@@ -46,6 +46,7 @@ _SIGS = {
     "tidar_verify_commit": (_i, [_vp, _vp, _i] + [_vp] * 4 + [_f] + [_vp] * 5 + [_i] * 9 + [_vp] * 12
                             + [_vp, _sz, _vp, _vp]),
     "tidar_testing_attn_step_stalled": (_i, [_vp] * 6 + [_i] * 6 + [_f, _i] + [_vp, _vp, _vp, ctypes.c_longlong, _vp]),
+    "tidar_testing_attn_splits": (_i, [_i] * 6),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -127,6 +128,11 @@ def tidar_testing_attn_step_stalled(q, k_new, v_new, k_cache, v_cache, prefix_le
     _check("tidar_testing_attn_step_stalled", _lib.tidar_testing_attn_step_stalled(
         _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(prefix_len), B, Hq, Hkv, D, k, P_max,
         softmax_scale, mask_mode, _ptr(out), _ptr(lse), _ptr(dev_status), wait_cycles, _stream(stream)))
+
+
+def tidar_testing_attn_splits(B, Hq, Hkv, D, k, P_max) -> int:
+    """Test hook (include/tidar_testing.h): the cluster size the attention launch would use (0: rejected sizes)."""
+    return _lib.tidar_testing_attn_splits(B, Hq, Hkv, D, k, P_max)
 
 
 def tidar_verify_workspace_size(B, k, V) -> int:

@@ -157,6 +157,12 @@ tidar_status tidar_testing_attn_step_stalled(const void *q, const void *k_new, c
                      out, lse, nullptr, 0, dev_status, stream, wait_cycles, 1);
 }
 
+int tidar_testing_attn_splits(int B, int Hq, int Hkv, int D, int k, int P_max) {
+    const AttnPlan pl = plan_attn(B, Hq, Hkv, D, k, P_max);
+    if (pl.status != TIDAR_OK) return 0;
+    return attn_sm100_pick_splits(D, (long)B * Hkv * pl.mtiles, pl.max_tiles);
+}
+
 size_t tidar_verify_workspace_size(int B, int k, int V) {
     if (B < 1 || k < 1 || k > kMaxDraft || V < 1 || V > kMaxVocab) return 0;
     return verify_workspace_bytes(B, k, V);

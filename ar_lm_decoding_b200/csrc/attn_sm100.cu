@@ -79,7 +79,12 @@ constexpr int TN = 128;
 constexpr int BOXR = 64;  // rows of one TMA box of a paged cache (one page): a tile is two boxes
 constexpr int STAGES = 3;
 constexpr int THREADS = 384;
-constexpr int kMaxSplits = 8;                        // cluster size limit (portable clusters)
+// Cluster sizes (key splits per row tile): 2..8, and the non-portable 9, 10, 12 and 15 where the device grants
+// them -- the larger sizes whose exchange blocks fit the region the portable ones need.
+constexpr int kMaxSplits = 15;
+__host__ __device__ constexpr bool split_count_ok(int S) {
+    return (S >= 1 && S <= 8) || S == 9 || S == 10 || S == 12 || S == 15;
+}
 constexpr long long kDrainCycles = kAttnWaitCycles;  // bound of the waits that drain issued work
 static_assert(BOXR == kPageRows, "a TMA box of the cache is one page");
 
@@ -97,7 +102,8 @@ __host__ __device__ constexpr int xchg_vals_bytes(int S, int D) { return (D / 8)
 __host__ __device__ constexpr int xchg_block_bytes(int S, int D) { return xchg_vals_bytes(S, D) + xchg_per(S) * 16; }
 constexpr int xchg_region_max(int D) {
     int m = 0;
-    for (int S = 2; S <= kMaxSplits; ++S) m = S * xchg_block_bytes(S, D) > m ? S * xchg_block_bytes(S, D) : m;
+    for (int S = 2; S <= kMaxSplits; ++S)
+        if (split_count_ok(S)) m = S * xchg_block_bytes(S, D) > m ? S * xchg_block_bytes(S, D) : m;
     return (m + 127) / 128 * 128;
 }
 constexpr int kStatsBytes = 4 * TM * 4;  // row statistics exchanged between the warpgroups (start of the ring)
@@ -127,7 +133,7 @@ static_assert(Smem<64>::STAGE_OFF + xchg_region_max(64) <= Smem<64>::BAR_OFF &&
 // the merge's per-row weights fit the row-statistics area: per rows x (S weights x 2 halves + 2)
 constexpr bool weights_fit() {
     for (int S = 2; S <= kMaxSplits; ++S)
-        if (xchg_per(S) * (2 * S + 2) * 4 > kStatsBytes) return false;
+        if (split_count_ok(S) && xchg_per(S) * (2 * S + 2) * 4 > kStatsBytes) return false;
     return true;
 }
 static_assert(weights_fit(), "merge weights larger than the row-statistics area");
@@ -308,7 +314,9 @@ __device__ __forceinline__ void split_tiles(int P, int R, int split, int n_split
     n = split < T ? (T - split + n_splits - 1) / n_splits : 0;
 }
 
-template <int D>
+// kLarge: the instantiation for the non-portable cluster sizes (more than 8 splits); the other one has only the
+// common sizes' merge, so the large sizes cost it no code.
+template <int D, bool kLarge>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_sm100_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tm_kc,
                       const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kn,
@@ -824,14 +832,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (warp == 0 && lane < S && lane != split) tc::mbar_arrive_remote(tc::cluster_map(sent, lane));
             const uint8_t *rv = smem + L::RECV_OFF;
             float *wts = reinterpret_cast<float *>(smem + L::KV_OFF);  // row-statistics area, free by now
-            switch (S) {
-                case 2: merge_rows<D, 2>(p, rv, wts, split, mt, b, kvh, tid); break;
-                case 3: merge_rows<D, 3>(p, rv, wts, split, mt, b, kvh, tid); break;
-                case 4: merge_rows<D, 4>(p, rv, wts, split, mt, b, kvh, tid); break;
-                case 5: merge_rows<D, 5>(p, rv, wts, split, mt, b, kvh, tid); break;
-                case 6: merge_rows<D, 6>(p, rv, wts, split, mt, b, kvh, tid); break;
-                case 7: merge_rows<D, 7>(p, rv, wts, split, mt, b, kvh, tid); break;
-                default: merge_rows<D, 8>(p, rv, wts, split, mt, b, kvh, tid); break;
+            if constexpr (kLarge) {
+                switch (S) {
+                    case 9: merge_rows<D, 9>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 10: merge_rows<D, 10>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 12: merge_rows<D, 12>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    default: merge_rows<D, 15>(p, rv, wts, split, mt, b, kvh, tid); break;
+                }
+            } else {
+                switch (S) {
+                    case 2: merge_rows<D, 2>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 3: merge_rows<D, 3>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 4: merge_rows<D, 4>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 5: merge_rows<D, 5>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 6: merge_rows<D, 6>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    case 7: merge_rows<D, 7>(p, rv, wts, split, mt, b, kvh, tid); break;
+                    default: merge_rows<D, 8>(p, rv, wts, split, mt, b, kvh, tid); break;
+                }
             }
         }
     }
@@ -900,8 +917,14 @@ cudaError_t launch(const AttnParams &p, cudaStream_t s) {
         !make_map(&qm, p.q, 3, dq, sq, bq))
         return cudaErrorInvalidValue;
     const int smem = Smem<D>::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const bool large = p.n_splits > 8;  // (chosen only where the occupancy query granted such clusters)
+    const auto kern = large ? attn_sm100_kernel<D, true> : attn_sm100_kernel<D, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    if (large) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.n_splits, p.Mpad / TM, p.B * p.Hkv);
     cfg.blockDim = dim3(THREADS, 1, 1);
@@ -916,7 +939,7 @@ cudaError_t launch(const AttnParams &p, cudaStream_t s) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, p, kc, vc, kn, vn, qm, q_tma);
+    e = cudaLaunchKernelEx(&cfg, kern, p, kc, vc, kn, vn, qm, q_tma);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -924,11 +947,16 @@ cudaError_t launch(const AttnParams &p, cudaStream_t s) {
 // Clusters of `S` CTAs of this kernel that can be resident at once (0 if the query fails).
 template <int D>
 int max_active_clusters(int S) {
-    static int cache[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+    static int cache[kMaxSplits + 1] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
     if (cache[S] >= 0) return cache[S];
     const int smem = Smem<D>::ALLOC;
-    if (cudaFuncSetAttribute(attn_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    const auto kern = S > 8 ? attn_sm100_kernel<D, true> : attn_sm100_kernel<D, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+    if (S > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        cudaGetLastError();
+        cache[S] = 0;
         return 0;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(S, 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
@@ -941,7 +969,7 @@ int max_active_clusters(int S) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_sm100_kernel<D>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
@@ -955,14 +983,15 @@ int attn_sm100_rows_per_tile() { return TM; }
 int attn_sm100_keys_per_tile() { return TN; }
 int attn_sm100_max_splits() { return kMaxSplits; }
 
-// Key splits per row tile (the cluster size): the largest S <= 8 and <= the
-// tile count for which all `groups` clusters are resident in one wave; 1 if
-// even single CTAs need several waves.
+// Key splits per row tile (the cluster size): the largest allowed S (split_count_ok) <= the tile count for which
+// all `groups` clusters are resident in one wave; 1 if even single CTAs need several waves.  Sizes above 8
+// (non-portable) only where the occupancy query grants them.
 int attn_sm100_pick_splits(int D, long groups, int max_tiles) {
-    const int hi = max(1, min(8, max_tiles));
+    const int hi = max(1, min(kMaxSplits, max_tiles));
     for (int S = hi; S > 1; --S) {
+        if (!split_count_ok(S)) continue;
         const int fit = D == 64 ? max_active_clusters<64>(S) : max_active_clusters<128>(S);
-        if (fit == 0 && S * groups <= kNumSMs) return S;  // query unavailable: assume one CTA per SM
+        if (fit == 0 && S <= 8 && S * groups <= kNumSMs) return S;  // query unavailable: one CTA per SM
         if (fit >= groups) return S;
     }
     return 1;

@@ -35,6 +35,15 @@ tidar_status tidar_testing_attn_step_stalled(const void *q, const void *k_new, c
                                              float softmax_scale, int mask_mode, void *out, float *lse,
                                              int32_t *dev_status, long long wait_cycles, void *stream);
 
+/*
+ * The cluster size (key splits per row tile) tidar_attn_step would use for
+ * these sizes on the current device (the largest that keeps every row tile's
+ * cluster resident in one wave; 1 when even single CTAs need several waves),
+ * or 0 for sizes tidar_attn_step rejects.  Queries the device's cluster
+ * occupancy; launches nothing.
+ */
+int tidar_testing_attn_splits(int B, int Hq, int Hkv, int D, int k, int P_max);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,20 @@ def test_full_size_every_row(name):
     assert eo <= O_TOL and el <= LSE_TOL, (name, eo, el)
 
 
+def test_split_choice():
+    """The cluster size each workload launches with: a supported size (2-8, or the non-portable 9, 10, 12, 15 the
+    device grants), never more splits than key tiles, and the whole grid in one wave unless it is a single split.
+    (test_full_size_every_row runs these same launch configurations against the oracle.)"""
+    from ar_lm_decoding_b200 import abi
+    for name, cfg in synth.CONFIGS.items():
+        S = abi.tidar_testing_attn_splits(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, cfg.P_max)
+        tiles = -(-cfg.P_max // 128) + -(-cfg.R // 128)
+        row_tiles = cfg.B * cfg.Hkv * -(-cfg.R * (cfg.Hq // cfg.Hkv) // 128)
+        assert S in (1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 12, 15) and S <= max(1, tiles), (name, S)
+        assert S == 1 or S * row_tiles <= 148, (name, S, row_tiles)
+    assert abi.tidar_testing_attn_splits(1, 4, 3, 128, 4, 100) == 0  # Hq not a multiple of Hkv: rejected
+
+
 def _plant_growing_spikes(cfg, inp, step_nat):
     """For every 128-key tile t of the cache and every KV head, overwrite one key so that it scores
     (4 + step_nat * t) natural-log units against one query row of that head's group (a different row each
