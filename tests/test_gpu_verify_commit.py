@@ -217,6 +217,29 @@ def test_verify_commit_many_sequences():
     assert len(report) <= 2
 
 
+@pytest.mark.parametrize("seed", range(12))
+def test_verify_commit_random_shapes(seed):
+    """Seeded random shapes through the fused call: batch 1-5 with ragged prefixes, k 1-16, an odd vocabulary size
+    (a last chunk of any length), bf16 or f32 logits, planted peaks or not, the trust mix on some seeds, 1-4 KV
+    heads, D 64 or 128, 1-2 layers; every output against the oracle's verify and commit."""
+    rng = np.random.default_rng(2000 + seed)
+    k = int(rng.integers(1, 17))
+    B = int(rng.integers(1, 6))
+    V = int(rng.integers(2, 60001 if k <= 8 else 20001))
+    cfg = synth.CONFIGS["tiny"].with_(B=B, k=k, V=V, Hq=4, Hkv=int(rng.choice([1, 2, 4])),
+                                      D=int(rng.choice([64, 128])), logits_dtype=str(rng.choice(["bf16", "f32"])),
+                                      peaks=bool(rng.integers(0, 2)), P=300, ragged=(0, 300), cfg_id=300 + seed)
+    trust_ar = 1.0 if seed % 3 else float(rng.choice([0.3, 0.6]))
+    inp = synth.make_verify_inputs(cfg, seed=seed)
+    kc, vc, kn, vn, pl, _, _, _, _ = _commit_inputs(cfg, seed, L=int(rng.integers(1, 3)))
+    got = _gpu().verify_commit(inp, kc, vc, kn, vn, pl, trust_ar=trust_ar)
+    report = []
+    _check_fused(inp, got, kc, vc, kn, vn, pl, report, trust_ar=trust_ar)
+    print(f"seed {seed}: B {B} k {k} V {V} {cfg.logits_dtype} peaks {cfg.peaks} lambda {trust_ar}: "
+          f"accept {got['accept_len'].tolist()}, exemptions {report}")
+    assert len(report) <= 1
+
+
 def test_verify_commit_bad_inputs():
     """A draft outside the vocabulary leaves its sequence untouched (no accept length); a prefix too close to
     the capacity keeps the verify outputs but skips that sequence's commit; the others are committed."""
