@@ -117,6 +117,30 @@ def test_paged_attention_equals_contiguous_and_oracle(case):
     assert np.abs(o - o_ref).max() <= O_TOL and np.abs(lse - lse_ref).max() <= LSE_TOL
 
 
+@pytest.mark.parametrize("seed", range(8))
+def test_paged_attention_random_shapes(seed):
+    """Seeded random shapes over randomly permuted pages: batch 1-4 with ragged prefixes (0 included), 1-4 KV heads,
+    group sizes 1-4, D 64 or 128, k 1-10; the same bits as the contiguous call and the oracle's results."""
+    rng = np.random.default_rng(3000 + seed)
+    Hkv = int(rng.choice([1, 2, 4]))
+    cfg = synth.CONFIGS["tiny"].with_(B=int(rng.integers(1, 5)), Hq=Hkv * int(rng.integers(1, 5)), Hkv=Hkv,
+                                      D=int(rng.choice([64, 128])), k=int(rng.integers(1, 11)),
+                                      ragged=(0, int(rng.integers(1, 1500))))
+    inp = synth.make_attn_inputs(cfg, seed=seed)
+    max_pages = cfg.P_max // PAGE
+    num_pages = cfg.B * max_pages + int(rng.integers(0, 9))
+    pool = Pool(1, num_pages, cfg.Hkv, cfg.D, cfg.B, max_pages, rng)
+    for b in range(cfg.B):
+        pool.write_rows(0, b, inp["k_cache"][b], inp["v_cache"][b], int(inp["prefix_len"][b]))
+    o, lse, st = _paged_attn(_bf16_dev(pool.k[0]), _bf16_dev(pool.v[0]), pool.table, inp, cfg, num_pages)
+    assert st == 0
+    import tidar_gpu
+    oc, lc = tidar_gpu.attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k)
+    assert np.array_equal(o, oc) and np.array_equal(lse, lc)
+    o_ref, lse_ref, _ = oracle.attn(inp, cfg.Hq, cfg.Hkv, cfg.D, cfg.k, dense=False)
+    assert np.abs(o - o_ref).max() <= O_TOL and np.abs(lse - lse_ref).max() <= LSE_TOL
+
+
 def test_paged_attention_bad_page_sets_status_and_skips():
     cfg = synth.CONFIGS["tiny"].with_(B=2, P=300)
     rng = np.random.default_rng(9)
