@@ -934,7 +934,8 @@ __global__ void __launch_bounds__(kStatThreads, 2) tail_kernel(const TailParams 
                 mx[x] = -INFINITY;
                 if (ib[x] < 0) continue;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) mx[x] = fmaxf(mx[x], item_val<MIX>(tr[x], qr[MIX ? x : 0], imix[x], p.lambda, e));
+                for (int e = 0; e < 32; ++e)
+                    mx[x] = fmaxf(mx[x], item_val<MIX>(tr[x], qr[MIX ? x : 0], imix[x], p.lambda, e));
                 // the thread that holds entry d of this row publishes that logit for the ratio test
                 const long long off = (long long)id[x] - (long long)ic[x] * kChunk;
                 if (off >= 0 && off < kChunk && (((int)off & 2047) >> 3) == tid) {
@@ -1029,7 +1030,8 @@ int resident_ctas() {
     static int n = -1;
     if (n >= 0) return n;
     int dev = 0, sms = 0, per = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, tail_kernel<MODE, DT, MIX>, kStatThreads, 0) != cudaSuccess) {
         cudaGetLastError();
         return 0;
