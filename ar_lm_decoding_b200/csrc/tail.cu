@@ -1032,7 +1032,8 @@ int resident_ctas() {
     int dev = 0, sms = 0, per = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, tail_kernel<MODE, DT, MIX>, kStatThreads, 0) != cudaSuccess) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, tail_kernel<MODE, DT, MIX>, kStatThreads, 0) !=
+            cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
