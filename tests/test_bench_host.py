@@ -102,3 +102,17 @@ def test_cpu_baseline_reports_single_thread_and_all_cores():
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
     assert cb["single_thread"]["threads"] == 1 and cb["single_thread"]["value"] > 0
     assert cb["host"]["nproc"] >= 1 and cb["host"]["cpu_model"]
+
+
+def test_copy_groups_cover_every_layer_once():
+    """The end-to-end leg's host-to-device copy groups: consecutive, covering layers 0..L-1 exactly once, sized
+    1, 2, 4, 8, 8, ... (the last takes the rest), never more than the cap."""
+    for L in (1, 2, 3, 7, 28, 36, 64, 80):
+        for cap in (1, 4, 8, 16):
+            groups = bench.copy_groups(L, cap=cap)
+            assert groups[0][0] == 0 and groups[-1][1] == L
+            assert all(a[1] == b[0] for a, b in zip(groups, groups[1:]))
+            sizes = [b - a for a, b in groups]
+            assert all(0 < s <= cap for s in sizes)
+            for i, s in enumerate(sizes[:-1]):
+                assert s == min(cap, 2 ** i)
