@@ -385,6 +385,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc::tma_prefetch_desc(&tm_vc);
         tc::tma_prefetch_desc(&tm_kn);
         tc::tma_prefetch_desc(&tm_vn);
+        // An L2 prefetch of this tile's Q rows, ahead of the wait: L2 is the point of coherence, so the copy
+        // after the wait still sees whatever the previous kernel writes there; the prefetch only starts the HBM
+        // read early.  (Several sequences without splits choose their sequence after the wait: no prefetch.)
+        if (q_tma && !(p.B > 1 && S == 1)) {
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+                tc::tma_prefetch_l2_3d(&tm_q, h * 64, kvh * p.G, b * p.R + mt * (TM / p.G));
+        }
     }
     if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
     // every global read below (prefix lengths, Q, K/V) waits for the previous kernel

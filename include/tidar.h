@@ -95,7 +95,7 @@ size_t tidar_attn_workspace_size(int B, int Hq, int Hkv, int D, int k, int P_max
  * k_new      bf16 [B, R, Hkv, D]  post-RoPE keys of this step's R tokens
  * v_new      bf16 [B, R, Hkv, D]
  * k_cache    bf16 [B, Hkv, P_max, D]  rows 0..P_b-1 are used; whole 128-row tiles
- *            are read (with a contiguous cache also up to 8 tiles from row 0
+ *            are read (with a contiguous cache also up to 15 tiles from row 0
  *            whatever P_b is), always inside the buffer, and rows past P_b are
  *            ignored, whatever they hold (NaN included)
  * v_cache    bf16 [B, Hkv, P_max, D]  (likewise)
